@@ -1,0 +1,278 @@
+"""Python binding of libsa: the four entry points with the C ABI's names.
+
+Argument marshalling only: tensors are passed to the C library as raw device
+pointers on torch's current stream, outputs and workspaces are allocated with
+torch when the caller does not pass them.  Every step of the computation runs
+in libsa's CUDA kernels; if the library is missing, ``_lib.load`` raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+from typing import Optional, Sequence
+
+import torch
+
+from . import _lib as L
+
+
+class SAError(RuntimeError):
+    def __init__(self, status: int, where: str, detail=None):
+        self.status = status
+        self.detail = detail
+        msg = "%s: %s" % (where, L.load().sa_status_string(status).decode())
+        if detail is not None:
+            msg += " (check %d, value %d)" % (detail[1], detail[2])
+        super().__init__(msg)
+
+
+def _check(status: int, where: str):
+    if status != L.SA_OK:
+        raise SAError(status, where)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream=None):
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def kv_struct(cache) -> L.KVCacheS:
+    """``cache``: any object with k, v, page_table, seq_lens tensors on the GPU
+    (k/v bf16 [num_pages][Hkv][P][d], page_table int32 [B][max_pages],
+    seq_lens int32 [B])."""
+    k, v = cache.k, cache.v
+    assert k.dtype == torch.bfloat16 and v.dtype == torch.bfloat16
+    assert k.is_contiguous() and v.is_contiguous() and k.shape == v.shape
+    pt, sl = cache.page_table, cache.seq_lens
+    assert pt.dtype == torch.int32 and sl.dtype == torch.int32 and pt.is_contiguous()
+    return L.KVCacheS(k.data_ptr(), v.data_ptr(), pt.data_ptr(), sl.data_ptr(), pt.shape[0], k.shape[1],
+                      k.shape[3], k.shape[2], pt.shape[1], k.shape[0])
+
+
+class Workspace:
+    """A reusable, zero-initialised device workspace (grows on demand)."""
+
+    def __init__(self, device=None):
+        self.device = device
+        self.buf: Optional[torch.Tensor] = None
+
+    def get(self, nbytes: int) -> torch.Tensor:
+        if self.buf is None or self.buf.numel() < nbytes:
+            n = max(nbytes, 256)
+            self.buf = torch.zeros(n + 256, dtype=torch.uint8, device=self.device or "cuda")
+        return self.buf
+
+    def aligned(self, nbytes: int):
+        buf = self.get(nbytes)
+        base = buf.data_ptr()
+        off = (-base) % 256
+        return ctypes.c_void_p(base + off), buf.numel() - off
+
+    def status(self, stream=None):
+        """Synchronise and return (status, detail) recorded by kernels (then cleared)."""
+        if self.buf is None:
+            return 0, (0, 0, 0)
+        ptr, _ = self.aligned(0)
+        det = (L.c_i32 * 3)()
+        st = L.load().sa_read_device_status(ptr, _stream(stream), det)
+        return st, tuple(det)
+
+    def raise_on_fault(self, where="device", stream=None):
+        st, det = self.status(stream)
+        if st != 0:
+            raise SAError(st, where, det)
+
+
+_default_ws = {}
+
+
+def _ws(ws: Optional[Workspace], device) -> Workspace:
+    if ws is not None:
+        return ws
+    key = str(device)
+    if key not in _default_ws:
+        _default_ws[key] = Workspace(device)
+    return _default_ws[key]
+
+
+def workspace_bytes(op: int, cache, num_q_heads=0, k=0, num_splits=0, num_tokens=0,
+                    block_args: Optional[L.BlockSelectArgsS] = None) -> int:
+    kv = kv_struct(cache)
+    q = L.WsQueryS(num_q_heads, k, num_splits, num_tokens,
+                   ctypes.pointer(block_args) if block_args is not None else None)
+    n = L.load().sa_workspace_bytes(op, ctypes.byref(kv), ctypes.byref(q))
+    if n == 0:
+        raise SAError(1, "sa_workspace_bytes")
+    return n
+
+
+def _qdtype(q: torch.Tensor) -> int:
+    if q.dtype == torch.float32:
+        return L.DTYPE_F32
+    if q.dtype == torch.bfloat16:
+        return L.DTYPE_BF16
+    raise TypeError("q must be fp32 or bf16")
+
+
+# --------------------------------------------------------------------------
+# selections
+# --------------------------------------------------------------------------
+@dataclasses.dataclass
+class TokenSelection:
+    idx: torch.Tensor     # int32 [B][Hq][k_cap]
+    count: torch.Tensor   # int32 [B][Hq]
+
+    def struct(self) -> L.SelectionS:
+        return L.SelectionS(L.SEL_TOKENS, self.idx.data_ptr(), self.count.data_ptr(), self.idx.shape[-1],
+                            None, None, 0)
+
+
+@dataclasses.dataclass
+class BlockSelection:
+    blocks: torch.Tensor        # int32 [B][max_blocks][4]
+    block_counts: torch.Tensor  # int32 [B]
+
+    def struct(self) -> L.SelectionS:
+        return L.SelectionS(L.SEL_BLOCKS, None, None, 0, self.blocks.data_ptr(),
+                            self.block_counts.data_ptr(), self.blocks.shape[1])
+
+
+@dataclasses.dataclass
+class BlockCSR:
+    row_ptr: torch.Tensor   # int32 [Hq*nQB + 1]
+    cols: torch.Tensor      # int32 [nnz_capacity]
+    tau: torch.Tensor       # fp32 [2][Hq] thresholds applied
+    num_q_heads: int
+    num_q_blocks: int
+
+
+# --------------------------------------------------------------------------
+# entry points
+# --------------------------------------------------------------------------
+def select_topk(cache, q: torch.Tensor, k: int, idx: Optional[torch.Tensor] = None,
+                count: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None,
+                stream=None) -> TokenSelection:
+    """Anchor-layer exact top-k per query head (``sa_select_topk``)."""
+    B, Hq, d = q.shape
+    dev = q.device
+    if idx is None:
+        idx = torch.empty((B, Hq, k), dtype=torch.int32, device=dev)
+    if count is None:
+        count = torch.empty((B, Hq), dtype=torch.int32, device=dev)
+    kv = kv_struct(cache)
+    w = _ws(ws, dev)
+    wp, wn = w.aligned(workspace_bytes(L.OP_SELECT_TOPK, cache, num_q_heads=Hq, k=k))
+    _check(L.load().sa_select_topk(ctypes.byref(kv), _ptr(q.contiguous()), _qdtype(q), Hq, k, _ptr(idx),
+                                   _ptr(count), wp, wn, _stream(stream)), "sa_select_topk")
+    return TokenSelection(idx, count)
+
+
+def sparse_decode_attn(cache, q: torch.Tensor, sel, scale: Optional[float] = None, num_splits: int = 1,
+                       out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                       want_lse: bool = True, ws: Optional[Workspace] = None, stream=None):
+    """Split-KV sparse decode + combine (``sa_sparse_decode_attn``).  Returns (out bf16, lse fp32)."""
+    B, Hq, d = q.shape
+    dev = q.device
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if out is None:
+        out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+    if lse is None and want_lse:
+        lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    kv = kv_struct(cache)
+    s = sel.struct()
+    w = _ws(ws, dev)
+    wp, wn = w.aligned(workspace_bytes(L.OP_DECODE, cache, num_q_heads=Hq, num_splits=num_splits))
+    _check(L.load().sa_sparse_decode_attn(ctypes.byref(kv), _ptr(q.contiguous()), _qdtype(q), Hq,
+                                          ctypes.byref(s), scale, num_splits, _ptr(out), _ptr(lse), wp, wn,
+                                          _stream(stream)), "sa_sparse_decode_attn")
+    return out, lse
+
+
+def select_blocks_spans(cache, spans: torch.Tensor, span_counts: torch.Tensor, span_round: torch.Tensor,
+                        max_blocks: Optional[int] = None, out: Optional[BlockSelection] = None,
+                        ws: Optional[Workspace] = None, stream=None) -> BlockSelection:
+    """Span masks -> page-segment block list (``sa_select_blocks``, mode SPANS).
+    spans int32 [B][max_spans][2], span_counts int32 [B], span_round uint8 [B][max_spans]."""
+    B = cache.page_table.shape[0]
+    dev = spans.device
+    if out is None:
+        mb = max_blocks if max_blocks is not None else cache.page_table.shape[1] + spans.shape[1]
+        out = BlockSelection(torch.empty((B, mb, 4), dtype=torch.int32, device=dev),
+                             torch.empty((B,), dtype=torch.int32, device=dev))
+    kv = kv_struct(cache)
+    a = L.BlockSelectArgsS()
+    a.mode = L.SEL_SPANS
+    a.spans, a.span_counts, a.span_round = spans.data_ptr(), span_counts.data_ptr(), span_round.data_ptr()
+    a.max_spans = spans.shape[1]
+    o = L.BlockListS()
+    o.blocks, o.block_counts, o.max_blocks = out.blocks.data_ptr(), out.block_counts.data_ptr(), out.blocks.shape[1]
+    w = _ws(ws, dev)
+    wp, wn = w.aligned(workspace_bytes(L.OP_SELECT_BLOCKS, cache, block_args=a))
+    _check(L.load().sa_select_blocks(ctypes.byref(kv), ctypes.byref(a), ctypes.byref(o), wp, wn,
+                                     _stream(stream)), "sa_select_blocks(spans)")
+    return out
+
+
+def select_blocks_rbs(cache, q: torch.Tensor, block_size: int = 64, scale: Optional[float] = None,
+                      tau_c=None, tau_r=None, p_c: float = 0.95, p_r: float = 0.97,
+                      force_diag: bool = True, force_first: bool = True,
+                      nnz_capacity: Optional[int] = None, out: Optional[BlockCSR] = None,
+                      ws: Optional[Workspace] = None, stream=None) -> BlockCSR:
+    """RBS two-branch block selection (``sa_select_blocks``, mode RBS).
+    Explicit thresholds: tau_c / tau_r fp32 [Hq] tensors (or floats);
+    otherwise quantile mode with p_c / p_r."""
+    T, Hq, d = q.shape
+    dev = q.device
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    nB = (T + block_size - 1) // block_size
+    if out is None:
+        cap = nnz_capacity if nnz_capacity is not None else Hq * nB * (nB + 1) // 2
+        out = BlockCSR(torch.empty(Hq * nB + 1, dtype=torch.int32, device=dev),
+                       torch.empty(max(cap, 1), dtype=torch.int32, device=dev),
+                       torch.empty((2, Hq), dtype=torch.float32, device=dev), Hq, nB)
+    tc = tr = None
+    if tau_c is not None:
+        tc = torch.as_tensor(tau_c, dtype=torch.float32, device=dev).expand(Hq).contiguous()
+        tr = torch.as_tensor(tau_r, dtype=torch.float32, device=dev).expand(Hq).contiguous()
+    kv = kv_struct(cache)
+    a = L.BlockSelectArgsS()
+    a.mode = L.SEL_RBS
+    a.q = q.data_ptr()
+    a.num_q_heads, a.num_tokens, a.block_size, a.scale = Hq, T, block_size, scale
+    a.tau_c = None if tc is None else tc.data_ptr()
+    a.tau_r = None if tr is None else tr.data_ptr()
+    a.p_c, a.p_r = p_c, p_r
+    a.force_diag, a.force_first = int(force_diag), int(force_first)
+    o = L.BlockListS()
+    o.row_ptr, o.cols, o.nnz_capacity = out.row_ptr.data_ptr(), out.cols.data_ptr(), out.cols.numel()
+    o.tau_out = out.tau.data_ptr()
+    w = _ws(ws, dev)
+    wp, wn = w.aligned(workspace_bytes(L.OP_SELECT_BLOCKS, cache, block_args=a))
+    _check(L.load().sa_select_blocks(ctypes.byref(kv), ctypes.byref(a), ctypes.byref(o), wp, wn,
+                                     _stream(stream)), "sa_select_blocks(rbs)")
+    return out
+
+
+def sparse_prefill_attn(cache, q: torch.Tensor, csr: BlockCSR, scale: Optional[float] = None,
+                        out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
+                        want_lse: bool = True, ws: Optional[Workspace] = None, stream=None):
+    """Causal block-sparse prefill (``sa_sparse_prefill_attn``).  Returns (out bf16, lse fp32)."""
+    T, Hq, d = q.shape
+    dev = q.device
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if out is None:
+        out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=dev)
+    if lse is None and want_lse:
+        lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+    kv = kv_struct(cache)
+    w = _ws(ws, dev)
+    wp, wn = w.aligned(workspace_bytes(L.OP_PREFILL, cache, num_q_heads=Hq, num_tokens=T))
+    _check(L.load().sa_sparse_prefill_attn(ctypes.byref(kv), _ptr(q), Hq, T, _ptr(csr.row_ptr),
+                                           _ptr(csr.cols), scale, 1, _ptr(out), _ptr(lse), wp, wn,
+                                           _stream(stream)), "sa_sparse_prefill_attn")
+    return out, lse

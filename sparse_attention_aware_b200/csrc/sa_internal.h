@@ -1,0 +1,118 @@
+// Internal launch interface between the C-ABI layer (sa_api.cu) and the
+// kernel translation units.  Not installed; not part of the ABI.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "sa.h"
+#include "sa_common.cuh"
+
+namespace sa {
+
+struct CacheArgs {
+    const uint16_t *k;
+    const uint16_t *v;
+    const int32_t *pt;
+    const int32_t *sl;
+    int B, Hkv, D, P, Plog2, max_pages, num_pages;
+};
+
+// ---- decode -----------------------------------------------------------------
+struct DecodeArgs {
+    CacheArgs c;
+    const void *q;
+    bool q_f32;
+    int Hq;
+    float qscale;  // scale * log2(e)
+    bool blocks;   // SA_SEL_BLOCKS
+    const int32_t *idx;
+    const int32_t *cnt;
+    int kcap;
+    const int32_t *ent;   // [B][max_blocks][4]
+    const int32_t *ecnt;  // [B]
+    int max_blocks;
+    int S;
+    float *part_o;   // [B*Hq][S][D]
+    float *part_ml;  // [B*Hq][S][2]
+    uint16_t *out;   // bf16 [B*Hq][D]
+    float *lse;      // [B*Hq] or null
+    DevStatus *st;
+};
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+
+// ---- top-k ------------------------------------------------------------------
+struct TopkArgs {
+    CacheArgs c;
+    const void *q;
+    bool q_f32;
+    int Hq;
+    int k;
+    float *scores;  // [B*Hq][Lcap]
+    int Lcap;
+    int32_t *idx;
+    int32_t *cnt;
+    DevStatus *st;
+};
+cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s);
+
+// ---- spans ------------------------------------------------------------------
+struct SpanArgs {
+    CacheArgs c;
+    const int32_t *spans;
+    const int32_t *span_counts;
+    const uint8_t *span_round;
+    int max_spans;
+    int32_t *ent;
+    int32_t *ecnt;
+    int max_blocks;
+    DevStatus *st;
+};
+cudaError_t launch_spans(const SpanArgs &a, cudaStream_t s);
+
+// ---- RBS selection ------------------------------------------------------------
+struct RbsArgs {
+    CacheArgs c;
+    const uint16_t *q;  // bf16 [T][Hq][D]
+    int Hq, T, bs, nB;
+    float scale;
+    const float *tau_c, *tau_r;  // explicit (device) or null
+    float p_c, p_r;
+    int force_diag, force_first;
+    // workspace pieces
+    float *cen;      // [Hkv][nB][D]
+    float *rad;      // [Hkv][nB]
+    float *qbar;     // [Hq][nB][D]
+    float *qnorm;    // [Hq][nB]
+    float *tau;      // [2][Hq] thresholds in use
+    uint32_t *bits;  // [Hq][nB][nB/32 words] mask bits
+    int words;       // words per row
+    int32_t *rowcnt; // [Hq*nB]
+    float *pair_sc;  // quantile mode: [Hq][nP] S_c, [Hq][nP] S_r
+    uint32_t *qhist; // quantile mode scratch
+    // outputs
+    int32_t *row_ptr;
+    int32_t *cols;
+    int64_t nnz_cap;
+    float *tau_out;
+    DevStatus *st;
+};
+size_t rbs_workspace_layout(int Hq, int Hkv, int D, int nB, bool quantile, size_t *offs);
+cudaError_t launch_rbs(const RbsArgs &a, cudaStream_t s);
+
+// ---- prefill ------------------------------------------------------------------
+struct PrefillArgs {
+    CacheArgs c;
+    const uint16_t *q;  // bf16 [T][Hq][128]
+    int Hq, T;
+    float scale;
+    const int32_t *row_ptr;
+    const int32_t *cols;
+    uint16_t *out;
+    float *lse;
+    int *work_counter;
+    DevStatus *st;
+};
+cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s);
+
+}  // namespace sa

@@ -1,0 +1,128 @@
+"""GPU parity: causal block-sparse prefill (tcgen05) against the fp64 oracle.
+
+Outputs within 2e-2 max-abs / 1e-2 mean-abs; LSE within 2e-3.  Masks: full
+causal, diagonal only, random CSR (with empty rows), and RBS-selected; token
+counts that leave a partial last block and an odd number of query blocks.
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import sparse_attention_aware_b200 as sa
+from sparse_attention_aware_b200 import workloads as W
+from tests.helpers import assert_close_attn, csr_to_mask, tau_in_gap
+
+pytestmark = pytest.mark.gpu
+
+
+def _mask_to_csr(mask, Hq, nB, dev):
+    rows, cols = [0], []
+    for h in range(Hq):
+        for i in range(nB):
+            sel = np.nonzero(mask[h, i * (i + 1) // 2: i * (i + 1) // 2 + i + 1])[0]
+            cols.extend(sel.tolist())
+            rows.append(len(cols))
+    rp = torch.tensor(rows, dtype=torch.int32, device=dev)
+    cl = torch.tensor(cols or [0], dtype=torch.int32, device=dev)
+    return sa.BlockCSR(rp, cl, torch.zeros((2, Hq), device=dev), Hq, nB)
+
+
+def _random_mask(seed, Hq, nB, density, empty_rows=0):
+    rng = np.random.default_rng(seed)
+    nP = nB * (nB + 1) // 2
+    m = (rng.random((Hq, nP)) < density).astype(np.uint8)
+    for h in range(Hq):
+        for i in range(nB):
+            if rng.random() < 0.5:
+                m[h, i * (i + 1) // 2 + i] = 1
+    for e in range(empty_rows):
+        h, i = int(rng.integers(Hq)), int(rng.integers(nB))
+        m[h, i * (i + 1) // 2: i * (i + 1) // 2 + i + 1] = 0
+    return m
+
+
+def _run(cuda_dev, wl, mask, rows=None):
+    T, Hq, d = wl.q.shape
+    nB = (T + 63) // 64
+    scale = 1 / math.sqrt(d)
+    csr = _mask_to_csr(mask, Hq, nB, cuda_dev)
+    ws = sa.Workspace(cuda_dev)
+    out, lse = sa.sparse_prefill_attn(wl.cache.to(cuda_dev), wl.q.to(cuda_dev), csr, scale, ws=ws)
+    ws.raise_on_fault()
+    ref, ref_lse = oracle.prefill(wl.cache, wl.q, 64, mask, scale, rows=rows)
+    g_out = out.float().cpu().numpy().reshape(-1, d)
+    g_lse = lse.cpu().numpy().reshape(-1)
+    if rows is not None:
+        g_out, g_lse = g_out[rows], g_lse[rows]
+    assert_close_attn(g_out, ref)
+    fin = np.isfinite(ref_lse)
+    assert np.all(np.isneginf(g_lse[~fin])) and np.all(g_out[~fin] == 0)
+    np.testing.assert_allclose(g_lse[fin], ref_lse[fin], atol=2e-3, rtol=0)
+    return out, lse
+
+
+@pytest.mark.parametrize("T,Hq,Hkv", [(640, 4, 2), (1000, 4, 4), (130, 2, 1), (64, 1, 1), (200, 8, 2)])
+def test_prefill_full_causal(cuda_dev, T, Hq, Hkv):
+    wl = W.random_prefill(300 + T, T, Hq, Hkv, 128, 64)
+    nB = (T + 63) // 64
+    _run(cuda_dev, wl, np.ones((Hq, nB * (nB + 1) // 2), dtype=np.uint8))
+
+
+@pytest.mark.parametrize("T", [640, 777])
+def test_prefill_diagonal_only_and_random(cuda_dev, T):
+    Hq, Hkv = 4, 2
+    wl = W.random_prefill(400 + T, T, Hq, Hkv, 128, 64)
+    nB = (T + 63) // 64
+    nP = nB * (nB + 1) // 2
+    diag = np.zeros((Hq, nP), dtype=np.uint8)
+    for i in range(nB):
+        diag[:, i * (i + 1) // 2 + i] = 1
+    _run(cuda_dev, wl, diag)
+    _run(cuda_dev, wl, _random_mask(T, Hq, nB, 0.3, empty_rows=3))
+
+
+def test_prefill_clustered_rbs_selection(cuda_dev):
+    """RBS-selected masks on clustered keys with outliers (large score range)."""
+    T, Hq, Hkv = 2048 + 64 * 3 + 17, 8, 2
+    wl = W.clustered_prefill(501, T=T, Hq=Hq, Hkv=Hkv, d=128, block=64, n_clusters=32)
+    scale = 1 / math.sqrt(128)
+    c, r = oracle.block_stats(wl.cache, 64)
+    qbar, qn = oracle.pool_q(wl.q, 64)
+    Sc, Sr = oracle.pair_scores(qbar, qn, c, r, scale)
+    tc = [tau_in_gap(Sc[h], 0.9)[0] for h in range(Hq)]
+    tr = [tau_in_gap(Sr[h], 0.93)[0] for h in range(Hq)]
+    mask = oracle.rbs_mask(Sc, Sr, tc, tr, True, True)
+    ws = sa.Workspace(cuda_dev)
+    gc = wl.cache.to(cuda_dev)
+    csr = sa.select_blocks_rbs(gc, wl.q.to(cuda_dev), 64, scale, tau_c=torch.tensor(tc), tau_r=torch.tensor(tr),
+                               ws=ws)
+    nB = (T + 63) // 64
+    rp = csr.row_ptr.cpu().numpy()
+    np.testing.assert_array_equal(csr_to_mask(rp, csr.cols.cpu().numpy()[: rp[-1]], Hq, nB), mask)
+    out, lse = sa.sparse_prefill_attn(gc, wl.q.to(cuda_dev), csr, scale, ws=ws)
+    ws.raise_on_fault()
+    ref, _ = oracle.prefill(wl.cache, wl.q, 64, mask, scale)
+    assert_close_attn(out.float().cpu().numpy().reshape(-1, 128), ref)
+    out2, lse2 = sa.sparse_prefill_attn(gc, wl.q.to(cuda_dev), csr, scale, ws=ws)
+    assert torch.equal(out, out2) and torch.equal(lse, lse2)
+
+
+def test_prefill_block_sparse_full_size_sampled(cuda_dev):
+    """32768 tokens, 32/4 heads, RBS-selected blocks; sampled query rows."""
+    wl = W.clustered_prefill(1004)
+    T, Hq, d = wl.q.shape
+    scale = 1 / math.sqrt(128)
+    c, r = oracle.block_stats(wl.cache, 64)
+    qbar, qn = oracle.pool_q(wl.q, 64)
+    Sc, Sr = oracle.pair_scores(qbar, qn, c, r, scale)
+    tc = [tau_in_gap(Sc[h], 0.95)[0] for h in range(Hq)]
+    tr = [tau_in_gap(Sr[h], 0.97)[0] for h in range(Hq)]
+    mask = oracle.rbs_mask(Sc, Sr, tc, tr, True, True)
+    rng = np.random.default_rng(5)
+    ts = np.concatenate([[0, 63, 64, 127, T - 1, T - 64], rng.integers(0, T, 250)])
+    hs = rng.integers(0, Hq, len(ts))
+    rows = (ts * Hq + hs).astype(np.int64)
+    _run(cuda_dev, wl, mask, rows=rows)
