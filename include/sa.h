@@ -241,17 +241,19 @@ SA_API sa_status sa_sparse_decode_attn(const sa_kv_cache *kv, const void *q, sa_
  * path).  Sequence 0 of `kv` holds the keys/values of the num_tokens prompt
  * tokens (page_size must equal the 64-token block).  For query token t of head
  * h in query block i = t / 64, attend to tokens t' <= t whose key block
- * t'/64 is listed in CSR row h*nQB + i (row_ptr/cols as produced by
- * sa_select_blocks(SA_SEL_RBS)).
+ * t'/64 is listed in CSR row h*nQB + i (csr->row_ptr / csr->cols /
+ * csr->nnz_capacity as produced by sa_select_blocks(SA_SEL_RBS); column
+ * entries at or past nnz_capacity, out of [0, i] or not strictly ascending are
+ * recorded as a device fault and skipped).
  *   q        bf16 [num_tokens][num_q_heads][128]
  *   out      bf16 [num_tokens][num_q_heads][128]
  *   lse_out  fp32 [num_tokens][num_q_heads] natural log, nullable
  *   causal   must be 1.
  */
 SA_API sa_status sa_sparse_prefill_attn(const sa_kv_cache *kv, const void *q, int32_t num_q_heads,
-                                 int32_t num_tokens, const int32_t *row_ptr, const int32_t *cols,
-                                 float scale, int32_t causal, void *out, float *lse_out, void *ws,
-                                 size_t ws_bytes, sa_stream_t stream);
+                                 int32_t num_tokens, const sa_block_list *csr, float scale,
+                                 int32_t causal, void *out, float *lse_out, void *ws, size_t ws_bytes,
+                                 sa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Workspace sizing, status                                                 */

@@ -73,7 +73,7 @@ def load(path: str = LIB_PATH):
     L.sa_select_blocks.argtypes = [P(KVCacheS), P(BlockSelectArgsS), P(BlockListS), c_vp, c_size, c_vp]
     L.sa_sparse_decode_attn.argtypes = [P(KVCacheS), c_vp, c_i32, c_i32, P(SelectionS), c_f32, c_i32,
                                         c_vp, c_vp, c_vp, c_size, c_vp]
-    L.sa_sparse_prefill_attn.argtypes = [P(KVCacheS), c_vp, c_i32, c_i32, c_vp, c_vp, c_f32, c_i32,
+    L.sa_sparse_prefill_attn.argtypes = [P(KVCacheS), c_vp, c_i32, c_i32, P(BlockListS), c_f32, c_i32,
                                          c_vp, c_vp, c_vp, c_size, c_vp]
     L.sa_workspace_bytes.argtypes = [c_i32, P(KVCacheS), P(WsQueryS)]
     L.sa_workspace_bytes.restype = c_size

@@ -270,9 +270,11 @@ def sparse_prefill_attn(cache, q: torch.Tensor, csr: BlockCSR, scale: Optional[f
     if lse is None and want_lse:
         lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
     kv = kv_struct(cache)
+    c = L.BlockListS()
+    c.row_ptr, c.cols, c.nnz_capacity = csr.row_ptr.data_ptr(), csr.cols.data_ptr(), csr.cols.numel()
     w = _ws(ws, dev)
     wp, wn = w.aligned(workspace_bytes(L.OP_PREFILL, cache, num_q_heads=Hq, num_tokens=T))
-    _check(L.load().sa_sparse_prefill_attn(ctypes.byref(kv), _ptr(q), Hq, T, _ptr(csr.row_ptr),
-                                           _ptr(csr.cols), scale, 1, _ptr(out), _ptr(lse), wp, wn,
-                                           _stream(stream)), "sa_sparse_prefill_attn")
+    _check(L.load().sa_sparse_prefill_attn(ctypes.byref(kv), _ptr(q), Hq, T, ctypes.byref(c), scale, 1,
+                                           _ptr(out), _ptr(lse), wp, wn, _stream(stream)),
+           "sa_sparse_prefill_attn")
     return out, lse

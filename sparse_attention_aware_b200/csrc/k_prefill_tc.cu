@@ -71,22 +71,30 @@ struct Merge {
     __device__ void init(const PrefillArgs &a, int r0, int lim_0, bool has1)
     {
         st = a.st;
+        // rows are read only inside [0, nnz_cap): a truncated (overflowed) CSR
+        // loses its tail entries, it never reads past the cols buffer
         const int b0 = __ldg(a.row_ptr + r0), e0 = __ldg(a.row_ptr + r0 + 1);
-        c0 = a.cols + b0;
+        c0 = a.cols + (b0 > 0 ? b0 : 0);
         n0 = e0 - b0;
         if (b0 < 0 || n0 < 0 || n0 > lim_0 + 1) {
             fault(st, CHK_CSR, r0);
             n0 = 0;
+        } else if ((long long)b0 + n0 > a.nnz_cap) {
+            fault(st, CHK_CSR, r0);
+            n0 = (long long)b0 >= a.nnz_cap ? 0 : (int)(a.nnz_cap - b0);
         }
         n1 = 0;
         c1 = c0;
         if (has1) {
             const int b1 = __ldg(a.row_ptr + r0 + 1), e1 = __ldg(a.row_ptr + r0 + 2);
-            c1 = a.cols + b1;
+            c1 = a.cols + (b1 > 0 ? b1 : 0);
             n1 = e1 - b1;
             if (b1 < 0 || n1 < 0 || n1 > lim_0 + 2) {
                 fault(st, CHK_CSR, r0 + 1);
                 n1 = 0;
+            } else if ((long long)b1 + n1 > a.nnz_cap) {
+                fault(st, CHK_CSR, r0 + 1);
+                n1 = (long long)b1 >= a.nnz_cap ? 0 : (int)(a.nnz_cap - b1);
             }
         }
         i0 = i1 = 0;

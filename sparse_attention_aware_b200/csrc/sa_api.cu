@@ -329,9 +329,9 @@ sa_status sa_select_blocks(const sa_kv_cache *kv, const sa_block_select_args *ar
 }
 
 sa_status sa_sparse_prefill_attn(const sa_kv_cache *kv, const void *q, int32_t num_q_heads,
-                                 int32_t num_tokens, const int32_t *row_ptr, const int32_t *cols,
-                                 float scale, int32_t causal, void *out, float *lse_out, void *ws,
-                                 size_t ws_bytes, sa_stream_t stream)
+                                 int32_t num_tokens, const sa_block_list *csr, float scale,
+                                 int32_t causal, void *out, float *lse_out, void *ws, size_t ws_bytes,
+                                 sa_stream_t stream)
 {
     PrefillArgs a{};
     sa_status st = check_cache(kv, &a.c);
@@ -343,7 +343,9 @@ sa_status sa_sparse_prefill_attn(const sa_kv_cache *kv, const void *q, int32_t n
     if (kv->batch < 1) return SA_ERR_INVALID_ARGUMENT;
     if ((long long)num_tokens > (long long)kv->max_pages_per_seq * kv->page_size) return SA_ERR_INVALID_ARGUMENT;
     if (!(scale == scale)) return SA_ERR_INVALID_ARGUMENT;
-    if (num_tokens > 0 && (!q || !row_ptr || !cols || !out)) return SA_ERR_INVALID_ARGUMENT;
+    if (num_tokens > 0 && (!q || !csr || !csr->row_ptr || !csr->cols || !out)) return SA_ERR_INVALID_ARGUMENT;
+    if (csr && csr->nnz_capacity < 0) return SA_ERR_INVALID_ARGUMENT;
+    if ((long long)kv->num_pages * kv->num_kv_heads * 64 >= (1LL << 31)) return SA_ERR_UNSUPPORTED;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(lse_out, 4)) return SA_ERR_INVALID_ARGUMENT;
     st = check_ws(ws, ws_bytes, ws_prefill());
     if (st != SA_OK) return st;
@@ -351,8 +353,10 @@ sa_status sa_sparse_prefill_attn(const sa_kv_cache *kv, const void *q, int32_t n
     a.Hq = num_q_heads;
     a.T = num_tokens;
     a.scale = scale;
-    a.row_ptr = row_ptr;
-    a.cols = cols;
+    if (num_tokens == 0) return SA_OK;
+    a.row_ptr = csr->row_ptr;
+    a.cols = csr->cols;
+    a.nnz_cap = csr->nnz_capacity;
     a.out = static_cast<uint16_t *>(out);
     a.lse = lse_out;
     a.work_counter = reinterpret_cast<int *>(static_cast<char *>(ws) + kHeader);

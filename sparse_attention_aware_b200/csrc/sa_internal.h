@@ -108,6 +108,7 @@ struct PrefillArgs {
     float scale;
     const int32_t *row_ptr;
     const int32_t *cols;
+    int64_t nnz_cap;
     uint16_t *out;
     float *lse;
     int *work_counter;

@@ -111,15 +111,18 @@ def test_host_validation_rejects_before_launch(lib):
     assert r == WS
     # prefill
     kv64 = _kv(P=64)
-    r = lib.sa_sparse_prefill_attn(ctypes.byref(kv), 0x70000, 8, 100, 0x80000, 0x90000, 0.1, 1, 0x60000,
-                                   None, 0x100000, 1 << 30, None)
-    assert r == UNS                                      # prefill needs 64-token pages
-    r = lib.sa_sparse_prefill_attn(ctypes.byref(kv64), 0x70000, 8, 100, 0x80000, 0x90000, 0.1, 0,
-                                   0x60000, None, 0x100000, 1 << 30, None)
-    assert r == UNS                                      # non-causal not built
-    r = lib.sa_sparse_prefill_attn(ctypes.byref(kv64), 0x70000, 8, 10_000, 0x80000, 0x90000, 0.1, 1,
-                                   0x60000, None, 0x100000, 1 << 30, None)
-    assert r == INV                                      # more tokens than the cache holds
+    csr = L.BlockListS()
+    csr.row_ptr, csr.cols, csr.nnz_capacity = 0x80000, 0x90000, 100
+    pre = lambda kvx, T, causal, c=csr: lib.sa_sparse_prefill_attn(
+        ctypes.byref(kvx), 0x70000, 8, T, ctypes.byref(c) if c is not None else None, 0.1, causal, 0x60000,
+        None, 0x100000, 1 << 30, None)
+    assert pre(kv, 100, 1) == UNS                        # prefill needs 64-token pages
+    assert pre(kv64, 100, 0) == UNS                      # non-causal not built
+    assert pre(kv64, 10_000, 1) == INV                   # more tokens than the cache holds
+    assert pre(kv64, 100, 1, None) == INV                # no CSR
+    bad = L.BlockListS()
+    bad.row_ptr, bad.cols, bad.nnz_capacity = 0x80000, 0x90000, -1
+    assert pre(kv64, 100, 1, bad) == INV
     # select_blocks
     a = L.BlockSelectArgsS()
     a.mode = 9
