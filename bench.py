@@ -1,0 +1,641 @@
+"""Benchmark of the head-aware sparse-attention hot path on B200.
+
+One step = one pass of every hot-path stage over one batch of seeded
+synthetic input, on the workload "block-sparse causal prefill at 131072
+tokens + Kascade decode at batch 32, context 65536":
+  * decode group: anchor top-k (scoring + radix select) over a 65536-token
+    paged cache (B=32, 32 q / 8 kv heads, d=128, 16-token shuffled pages),
+    k=4096 per query head, then split-KV decode (8 splits) + combine on the
+    anchor layer and 3 reuse layers (fresh Q and V, anchor K);
+  * masked decode: one DA/LoZA step on a 131072-token cache (B=4, 64 q / 8 kv
+    heads): span lists -> page segments -> split-KV decode + combine;
+  * prefill: RBS selection (block stats, pooled queries, pair scores,
+    per-head quantile thresholds, OR, CSR) and tcgen05 block-sparse causal
+    prefill over T=131072 tokens (32 q / 4 kv heads, 64x64 blocks), with
+    quantile levels calibrated once so the kept block density is ~5%.
+
+Headline value: decode-group algorithmic GB/s (selected K/V rows + anchor K
+scan + indices + Q/O + page table) / decode-group device time.  Also
+reported: prefill TFLOP/s on selected tiles, roofline fractions against the
+measured peaks, the CPU oracle on a bounded sample, and an end-to-end number
+through the public API with host buffers.
+
+Usage:  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "sparse decode GB/s & % HBM peak; block-sparse prefill TFLOPS at 128K (1 B200)"
+WORKLOAD = "block-sparse causal prefill T=131072 (32q/4kv, d=128, 64x64 blocks, ~5% density) + " \
+           "Kascade decode B=32 L=65536 (32q/8kv, top-k 4096, anchor + 3 reuse, 8 splits)"
+TILE_FLOPS = 4 * 64 * 64 * 128
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+# kernels each API call launches (libsa)
+LAUNCHES = {"select_topk": 2, "decode": 2, "spans": 1, "rbs_quantile": 8, "prefill": 1}
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return {k: float(d[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")}, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# workload
+# ---------------------------------------------------------------------------
+class Cfg:
+    def __init__(self, small=False):
+        if small:   # quick variant for profiling captures
+            self.dec = dict(B=8, Hq=32, Hkv=8, d=128, L=32768, P=16, k=2048, layers=4, splits=8)
+            self.pre = dict(T=32768, Hq=32, Hkv=4, d=128, block=64)
+            self.msk = dict(B=4, Hq=64, Hkv=8, d=128, L=32768, P=16)
+        else:
+            self.dec = dict(B=32, Hq=32, Hkv=8, d=128, L=65536, P=16, k=4096, layers=4, splits=8)
+            self.pre = dict(T=131072, Hq=32, Hkv=4, d=128, block=64)
+            self.msk = dict(B=4, Hq=64, Hkv=8, d=128, L=131072, P=16)
+        self.small = small
+        self.density_target = 0.05
+
+
+def decode_group_bytes(c):
+    B, Hq, Hkv, d, L, k, layers = c["B"], c["Hq"], c["Hkv"], c["d"], c["L"], c["k"], c["layers"]
+    row = d * 2
+    pt = B * (L // c["P"]) * 4
+    scan = B * Hkv * L * row + B * Hq * d * 2 + pt + B * Hq * k * 4      # anchor K scan, Q, pages, idx write
+    per_layer = B * Hq * k * 2 * row + B * Hq * k * 4 + 2 * B * Hq * d * 2 + pt   # K+V rows, idx, Q, O
+    return scan + layers * per_layer
+
+
+def build(cfg, dev, seed=1005):
+    import torch
+    from sparse_attention_aware_b200 import workloads as W
+    c = cfg.dec
+    dec = W.gqa_decode(seed, device=dev, B=c["B"], Hq=c["Hq"], Hkv=c["Hkv"], d=c["d"], L=c["L"], P=c["P"],
+                       k=c["k"], layers=c["layers"], num_splits=c["splits"])
+    p = cfg.pre
+    pre = W.clustered_prefill(seed, device=dev, T=p["T"], Hq=p["Hq"], Hkv=p["Hkv"], d=p["d"], block=p["block"])
+    m = cfg.msk
+    msk = W.masked_decode(1003, device=dev, B=m["B"], Hq=m["Hq"], Hkv=m["Hkv"], d=m["d"], L=m["L"], P=m["P"],
+                          steps=64)
+    torch.cuda.synchronize(dev)
+    return dec, pre, msk
+
+
+def calibrate_density(pre, ws, target=0.05, tol=0.0025):
+    """Quantile level p_c (p_r = p_c + 0.02) with kept block density ~target,
+    found by bisection with the GPU selector on this seed."""
+    import sparse_attention_aware_b200 as sa
+    T, Hq, d = pre.q.shape
+    nB = (T + 63) // 64
+    total = Hq * nB * (nB + 1) // 2
+    lo, hi = 0.80, 0.999
+    best = None
+    for _ in range(14):
+        pc = 0.5 * (lo + hi)
+        pr = min(pc + 0.02, 1.0)
+        csr = sa.select_blocks_rbs(pre.cache, pre.q, 64, 1 / math.sqrt(d), p_c=pc, p_r=pr, ws=ws)
+        dens = int(csr.row_ptr[-1]) / total
+        best = (pc, pr, dens)
+        if abs(dens - target) <= tol * 0.5:
+            break
+        if dens > target:
+            lo = pc
+        else:
+            hi = pc
+    return best
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    Q = ("index,pci.bus_id,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id=None):
+        self.bus_id = str(bus_id or "").lower()
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.Q, "--format=csv,noheader,nounits",
+                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                         text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        rows = []
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 10:
+                continue
+            if self.bus_id and not f[1].lower().endswith(self.bus_id):
+                continue
+            rows.append(f)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[2]) for r in rows]
+        mx = float(rows[0][3])
+        loaded = [s for s in sm if s > 0.5 * mx] or sm
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for i, n in enumerate(names):
+                if r[6 + i].lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(rows), "power_w_max": max(float(r[4]) for r in rows)}
+
+
+# ---------------------------------------------------------------------------
+# one step
+# ---------------------------------------------------------------------------
+class Step:
+    def __init__(self, cfg, dec, pre, msk, pc, pr, dev):
+        import torch
+        import sparse_attention_aware_b200 as sa
+        from sparse_attention_aware_b200 import spans as SP
+        self.sa, self.torch, self.SP = sa, torch, SP
+        self.cfg, self.dec, self.pre, self.msk, self.pc, self.pr, self.dev = cfg, dec, pre, msk, pc, pr, dev
+        self.ws = [sa.Workspace(dev) for _ in range(4)]
+        c = cfg.dec
+        self.scale_dec = 1 / math.sqrt(c["d"])
+        B, Hq, d = c["B"], c["Hq"], c["d"]
+        self.idx = torch.empty((B, Hq, c["k"]), dtype=torch.int32, device=dev)
+        self.cnt = torch.empty((B, Hq), dtype=torch.int32, device=dev)
+        self.outs = [torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev) for _ in range(c["layers"])]
+        self.lses = [torch.empty((B, Hq), dtype=torch.float32, device=dev) for _ in range(c["layers"])]
+        self.caches = [dec.cache.with_v(v) for v in dec.v_layers]
+        T, Hqp, dp = pre.q.shape
+        nB = (T + 63) // 64
+        self.nB = nB
+        cap = int(Hqp * nB * (nB + 1) // 2 * 0.12) + Hqp * nB * 2
+        self.csr = sa.BlockCSR(torch.empty(Hqp * nB + 1, dtype=torch.int32, device=dev),
+                               torch.empty(cap, dtype=torch.int32, device=dev),
+                               torch.empty((2, Hqp), dtype=torch.float32, device=dev), Hqp, nB)
+        self.pout = torch.empty((T, Hqp, dp), dtype=torch.bfloat16, device=dev)
+        self.plse = torch.empty((T, Hqp), dtype=torch.float32, device=dev)
+        m = cfg.msk
+        self.mout = torch.empty((m["B"], m["Hq"], m["d"]), dtype=torch.bfloat16, device=dev)
+        self.mlse = torch.empty((m["B"], m["Hq"]), dtype=torch.float32, device=dev)
+        self.mblk = sa.BlockSelection(torch.empty((m["B"], m["L"] // m["P"] + 8, 4), dtype=torch.int32, device=dev),
+                                      torch.empty((m["B"],), dtype=torch.int32, device=dev))
+        # span lists for every masked-decode step, packed once (host-side DA/LoZA state)
+        self.span_t = []
+        for s in range(msk.q_steps.shape[0]):
+            lists = []
+            for b in range(m["B"]):
+                mode = SP.MODE_IDS[int(msk.modes[s, b])]
+                lists.append(SP.spans_for(mode, m["L"], msk.chunk, msk.origin, msk.focus_chunks[s, b].tolist()))
+            self.span_t.append(SP.pack(lists, dev, max_spans=2))
+        self.mstep = 0
+        self.masked_tokens = []
+        for s in range(msk.q_steps.shape[0]):
+            tot = 0
+            for b in range(m["B"]):
+                mode = SP.MODE_IDS[int(msk.modes[s, b])]
+                if mode == SP.STREAMING:
+                    tot += 4 + 1024
+                elif mode == SP.LOCAL:
+                    tot += 512
+                else:
+                    tot += 2 * msk.chunk
+            self.masked_tokens.append(tot)
+
+    # parts --------------------------------------------------------------
+    def decode_group(self, q_layers):
+        sa = self.sa
+        c = self.cfg.dec
+        sel = sa.select_topk(self.caches[0], q_layers[0], c["k"], idx=self.idx, count=self.cnt, ws=self.ws[0])
+        for li in range(c["layers"]):
+            sa.sparse_decode_attn(self.caches[li], q_layers[li], sel, self.scale_dec, c["splits"],
+                                  out=self.outs[li], lse=self.lses[li], ws=self.ws[0])
+        return self.outs
+
+    def masked_decode(self, q):
+        sa = self.sa
+        s = self.mstep % len(self.span_t)
+        spans, cnt, rnd = self.span_t[s]
+        blk = sa.select_blocks_spans(self.msk.cache, spans, cnt, rnd, out=self.mblk, ws=self.ws[1])
+        sa.sparse_decode_attn(self.msk.cache, q, blk, 1 / math.sqrt(q.shape[-1]), 8, out=self.mout, lse=self.mlse,
+                              ws=self.ws[1])
+        return self.mout
+
+    def rbs_select(self, q):
+        d = q.shape[-1]
+        return self.sa.select_blocks_rbs(self.pre.cache, q, 64, 1 / math.sqrt(d), p_c=self.pc, p_r=self.pr,
+                                         out=self.csr, ws=self.ws[2])
+
+    def prefill(self, q, csr):
+        d = q.shape[-1]
+        return self.sa.sparse_prefill_attn(self.pre.cache, q, csr, 1 / math.sqrt(d), out=self.pout, lse=self.plse,
+                                           ws=self.ws[3])
+
+    def launches_per_step(self):
+        L = LAUNCHES
+        return (L["select_topk"] + self.cfg.dec["layers"] * L["decode"] + L["spans"] + L["decode"]
+                + L["rbs_quantile"] + L["prefill"])
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=40)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--small", action="store_true", help="smaller workload (profiling captures)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return reference_arm(args)
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    import sparse_attention_aware_b200 as sa
+    from sparse_attention_aware_b200 import _lib
+    _lib.load()
+
+    cfg = Cfg(small=args.small)
+    dec, pre, msk = build(cfg, dev)
+    cal_ws = sa.Workspace(dev)
+    pc, pr, density = calibrate_density(pre, cal_ws, cfg.density_target)
+    step = Step(cfg, dec, pre, msk, pc, pr, dev)
+    # selected tiles / executed (super-block union) tiles of the prefill
+    csr = step.rbs_select(pre.q)
+    torch.cuda.synchronize()
+    sel_tiles = int(csr.row_ptr[-1])
+    exec_tiles = union_tiles(csr, pre.q.shape[1], step.nB)
+
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+
+    def run_step(timed=None):
+        e = [ev() for _ in range(5)] if timed is not None else None
+        if e: e[0].record(stream)
+        step.decode_group(dec.q_layers)
+        if e: e[1].record(stream)
+        q = msk.q_steps[step.mstep % msk.q_steps.shape[0]]
+        step.masked_decode(q)
+        if e: e[2].record(stream)
+        c = step.rbs_select(pre.q)
+        if e: e[3].record(stream)
+        step.prefill(pre.q, c)
+        if e: e[4].record(stream)
+        step.mstep += 1
+        if timed is not None:
+            timed.append(e)
+
+    W_steps = max(args.warmup, 3)
+    for _ in range(W_steps):
+        run_step()
+    torch.cuda.synchronize()
+    for w in step.ws + [cal_ws]:
+        w.raise_on_fault("warm-up")
+
+    bus = None
+    try:
+        pr_ = torch.cuda.get_device_properties(dev)
+        bus = "%02x:%02x.0" % (int(pr_.pci_bus_id), int(pr_.pci_device_id))
+    except Exception:
+        pass
+    clocks = ClockSampler(bus)
+    clocks.start()
+    time.sleep(0.3)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t_start, t_end = ev(), ev()
+    evs = []
+    t_start.record(stream)
+    for _ in range(args.steps):
+        run_step(evs)
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    for w in step.ws:
+        w.raise_on_fault("timed region")
+
+    total_ms = t_start.elapsed_time(t_end)
+    parts = {"decode": 0.0, "masked": 0.0, "rbs_select": 0.0, "prefill": 0.0}
+    for e in evs:
+        parts["decode"] += e[0].elapsed_time(e[1])
+        parts["masked"] += e[1].elapsed_time(e[2])
+        parts["rbs_select"] += e[2].elapsed_time(e[3])
+        parts["prefill"] += e[3].elapsed_time(e[4])
+    K = args.steps
+    vals = torch.tensor([total_ms, parts["decode"], parts["masked"], parts["rbs_select"], parts["prefill"]],
+                        dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    total_ms, dec_ms, msk_ms, rbs_ms, pre_ms = [float(x) for x in vals.tolist()]
+
+    dec_bytes = decode_group_bytes(cfg.dec)
+    m = cfg.msk
+    msk_bytes = sum(step.masked_tokens[s % len(step.masked_tokens)] for s in range(K)) * m["Hkv"] * m["d"] * 2 * 2 \
+        + K * 2 * m["B"] * m["Hq"] * m["d"] * 2
+    p = cfg.pre
+    T, Hqp, dp = p["T"], p["Hq"], p["d"]
+    pre_flops = sel_tiles * TILE_FLOPS
+    rbs_bytes = T * p["Hkv"] * dp * 2 + T * Hqp * dp * 2 + (Hqp * step.nB + 1 + sel_tiles) * 4
+
+    pk, pk_kind = peaks()
+    dec_gbs = world * K * dec_bytes / (dec_ms * 1e-3) / 1e9
+    pre_tflops = world * K * pre_flops / (pre_ms * 1e-3) / 1e12
+    per_gpu_dec = dec_gbs / world
+    per_gpu_pre = pre_tflops / world
+
+    result = {
+        "metric": METRIC, "value": round(dec_gbs, 2), "unit": "GB/s", "n_gpus": world, "steps": K,
+        "warmup": W_steps, "ms_per_step": round(total_ms / K, 4), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16 in / fp32 accumulate",
+        "data": "synthetic (seeded; shapes and laws of the pages' workloads)",
+        "config": {"workload": WORKLOAD + (" [small variant]" if cfg.small else ""),
+                   "decode": cfg.dec, "prefill": dict(cfg.pre, p_c=round(pc, 5), p_r=round(pr, 5),
+                                                      block_density=round(density, 5)),
+                   "masked_decode": cfg.msk, "parallelism": "dp%d (independent replicas)" % world,
+                   "l2": "inputs larger than L2 (decode K cache %.1f GB, prefill Q %.2f GB)"
+                         % (cfg.dec["B"] * cfg.dec["Hkv"] * cfg.dec["L"] * 256 / 1e9, T * Hqp * dp * 2 / 1e9)},
+        "decode": {"gbs": round(dec_gbs, 2), "frac_hbm": round(per_gpu_dec / pk["hbm_gbs"], 4),
+                   "ms_per_group": round(dec_ms / K, 4), "bytes_per_group": dec_bytes,
+                   "tokens_per_s": round(world * K * cfg.dec["B"] / (dec_ms * 1e-3), 1)},
+        "prefill": {"tflops": round(pre_tflops, 2), "frac_bf16_sustained": round(per_gpu_pre / pk["bf16_tflops_sustained"], 4),
+                    "frac_bf16_burst": round(per_gpu_pre / pk["bf16_tflops"], 4),
+                    "ms": round(pre_ms / K, 4), "selected_tiles": sel_tiles, "executed_tiles": exec_tiles,
+                    "tokens_per_s": round(world * K * T / (pre_ms * 1e-3), 1)},
+        "rbs_select": {"ms": round(rbs_ms / K, 4), "gbs": round(world * K * rbs_bytes / (rbs_ms * 1e-3) / 1e9, 2),
+                       "frac_hbm": round(K * rbs_bytes / (rbs_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
+        "masked_decode": {"ms_per_step": round(msk_ms / K, 4),
+                          "gbs": round(world * msk_bytes / (msk_ms * 1e-3) / 1e9, 2),
+                          "frac_hbm": round(msk_bytes / (msk_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
+        "roofline": {"bound": "tensor", "kernel": "k_prefill_tc", "achieved": round(per_gpu_pre, 2),
+                     "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": round(per_gpu_pre / pk["bf16_tflops_sustained"], 4), "traffic": None,
+                     "peak_source": "%s bf16_tflops_sustained (kernel timed inside a multi-kernel step)" % pk_kind,
+                     "algorithmic": "selected tiles x 4*64*64*128 FLOP per launch; CUDA events around the launch"},
+        "roofline_decode": {"bound": "hbm", "kernel": "k_topk_score + k_decode_split + combine",
+                            "achieved": round(per_gpu_dec, 2), "peak": pk["hbm_gbs"], "unit": "GB/s",
+                            "frac": round(per_gpu_dec / pk["hbm_gbs"], 4), "traffic": None,
+                            "peak_source": "%s hbm_gbs" % pk_kind},
+        "clocks": clk,
+        "gpu_launches": step.launches_per_step() * K,
+    }
+    traffic = load_traffic()
+    if traffic:
+        result["roofline"]["traffic"] = traffic.get("k_prefill_tc")
+        result["roofline_decode"]["traffic"] = traffic.get("decode")
+
+    if not args.no_e2e:
+        result["e2e"] = e2e(step, dec, pre, msk, cfg, args, world, dev, dist if world > 1 else None)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        result["cpu_baseline"] = cpu_baseline(cfg, dec, pre, pc, pr)
+    if rank == 0:
+        print(json.dumps(result))
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def load_traffic():
+    """Per-launch DRAM bytes (read + write) from the committed ncu summary, if
+    it matches the current kernels; None otherwise."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        with open(p) as f:
+            return json.load(f)
+    except Exception:
+        return None
+
+
+def union_tiles(csr, Hq, nB):
+    """Key tiles the prefill kernel executes: per 128-row super-block, the
+    union of its two CSR rows."""
+    import numpy as np
+    rp = csr.row_ptr.cpu().numpy().astype(np.int64)
+    cols = csr.cols[: int(rp[-1])].cpu().numpy()
+    tot = 0
+    for h in range(Hq):
+        for I in range((nB + 1) // 2):
+            r0 = h * nB + 2 * I
+            a = cols[rp[r0]:rp[r0 + 1]]
+            if 2 * I + 1 < nB:
+                b = cols[rp[r0 + 1]:rp[r0 + 2]]
+                tot += len(np.union1d(a, b))
+            else:
+                tot += len(a)
+    return int(tot)
+
+
+def e2e(step, dec, pre, msk, cfg, args, world, dev, dist):
+    """The same metric through the public API with host buffers: every step
+    copies its inputs (queries of every decode layer, the masked-decode query,
+    the prompt's Q) from pinned host memory and reads the outputs (attention
+    outputs and LSEs) back; KV caches stay resident as a serving engine's do."""
+    import torch
+    qh = [q.cpu().pin_memory() for q in dec.q_layers]
+    mq = msk.q_steps.cpu().pin_memory()
+    pq = pre.q.cpu().pin_memory()
+    outs_h = [torch.empty_like(o, device="cpu").pin_memory() for o in step.outs]
+    mo_h = torch.empty_like(step.mout, device="cpu").pin_memory()
+    po_h = torch.empty_like(step.pout, device="cpu").pin_memory()
+    qd = [torch.empty_like(q, device=dev) for q in dec.q_layers]
+    mqd = torch.empty_like(msk.q_steps[0])
+    pqd = torch.empty_like(pre.q)
+    h2d = sum(q.numel() * q.element_size() for q in qh) + mq[0].numel() * 2 + pq.numel() * 2
+    d2h = sum(o.numel() * 2 for o in outs_h) + mo_h.numel() * 2 + po_h.numel() * 2
+    stream = torch.cuda.current_stream()
+    ev = lambda: torch.cuda.Event(enable_timing=True)
+    K = args.steps
+
+    def one(evs=None):
+        e = [ev() for _ in range(3)] if evs is not None else None
+        if e: e[0].record(stream)
+        for i in range(len(qh)):
+            qd[i].copy_(qh[i], non_blocking=True)
+        outs = step.decode_group(qd)
+        for i, o in enumerate(outs):
+            outs_h[i].copy_(o, non_blocking=True)
+        mqd.copy_(mq[step.mstep % mq.shape[0]], non_blocking=True)
+        mo_h.copy_(step.masked_decode(mqd), non_blocking=True)
+        if e: e[1].record(stream)
+        pqd.copy_(pq, non_blocking=True)
+        out, _ = step.prefill(pqd, step.rbs_select(pqd))
+        po_h.copy_(out, non_blocking=True)
+        if e: e[2].record(stream)
+        step.mstep += 1
+        if evs is not None:
+            evs.append(e)
+
+    one()
+    torch.cuda.synchronize()
+    evs = []
+    for _ in range(K):
+        one(evs)
+    torch.cuda.synchronize()
+    dec_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
+    pre_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
+    vals = torch.tensor([dec_ms, pre_ms], dtype=torch.float64, device=dev)
+    if dist is not None:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    dec_ms, pre_ms = [float(x) for x in vals.tolist()]
+    dec_bytes = decode_group_bytes(cfg.dec)
+    csr_tiles = int(step.csr.row_ptr[-1])
+    return {"value": round(world * K * dec_bytes / (dec_ms * 1e-3) / 1e9, 2), "unit": "GB/s",
+            "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h),
+            "prefill_tflops": round(world * K * csr_tiles * TILE_FLOPS / (pre_ms * 1e-3) / 1e12, 2),
+            "note": "decode value includes the masked-decode step's copies; prefill includes Q in / O out"}
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle (bounded sample)
+# ---------------------------------------------------------------------------
+def _sub_decode(dec, bsel, dev_out="cpu"):
+    """The decode workload restricted to sequences bsel, pages gathered into a
+    compact host cache (same values, same page structure)."""
+    import torch
+    from sparse_attention_aware_b200 import workloads as W
+    c = dec.cache
+    pt = c.page_table[bsel].long()
+    used = pt.reshape(-1)
+    new_pt = torch.arange(used.numel(), dtype=torch.int32).reshape(pt.shape)
+    k = c.k[used].to(dev_out)
+    vs = [v[used].to(dev_out) for v in dec.v_layers]
+    cache = W.PagedCache(k, vs[0], new_pt, c.seq_lens[bsel].cpu())
+    qs = [q[bsel].cpu() for q in dec.q_layers]
+    return cache, vs, qs
+
+
+def cpu_baseline(cfg, dec, pre, pc, pr, budget_s=10.0):
+    """The oracle, as it stands, on the host cores: anchor top-k + 4 decode
+    layers for pairs of sequences (all heads) until about budget_s seconds of
+    oracle time, and RBS selection + block-sparse prefill for one head on 256
+    sampled query rows.  Reported in the metric's unit (decode GB/s on the
+    sample's algorithmic bytes)."""
+    import numpy as np
+    import oracle
+    c = cfg.dec
+    B = int(dec.cache.page_table.shape[0])
+    scale = 1 / math.sqrt(c["d"])
+    t_dec, nseq = 0.0, 0
+    while nseq < B and t_dec < budget_s:
+        bsel = list(range(nseq, min(nseq + 2, B)))
+        cache, vs, qs = _sub_decode(dec, bsel)
+        cv = oracle.CacheView(cache)
+        t0 = time.time()
+        idx, cnt = oracle.select_topk(cv, qs[0], c["k"])
+        for li in range(c["layers"]):
+            oracle.decode_tokens(oracle.CacheView(cache.with_v(vs[li])), qs[li], idx, cnt, scale)
+        t_dec += time.time() - t0
+        nseq += len(bsel)
+    dec_gbs = decode_group_bytes(dict(c, B=nseq)) / t_dec / 1e9
+    # prefill sample: one head's selection + 256 query rows
+    from sparse_attention_aware_b200 import workloads as W
+    T = int(pre.q.shape[0])
+    pc_ = pre.cache
+    cpre = W.PagedCache(pc_.k[:, :1].contiguous().cpu(), pc_.v[:, :1].contiguous().cpu(),
+                        pc_.page_table.cpu(), pc_.seq_lens.cpu())      # kv head 0 only
+    q = pre.q[:, :1].contiguous().cpu()                                # its first query head
+    t1 = time.time()
+    cs, rs = oracle.block_stats(cpre, 64)
+    qb, qn = oracle.pool_q(q, 64)
+    Sc, Sr = oracle.pair_scores(qb, qn, cs, rs, 1 / math.sqrt(128))
+    tc, tr = oracle.quantile(Sc[0], pc), oracle.quantile(Sr[0], pr)
+    mask = oracle.rbs_mask(Sc, Sr, [tc], [tr], True, True)
+    rng = np.random.default_rng(0)
+    rows = np.sort(rng.integers(0, T, 256)).astype(np.int64)
+    oracle.prefill(cpre, q, 64, mask, 1 / math.sqrt(128), rows=rows)
+    t_pre = time.time() - t1
+    flops = 0
+    for t in rows:
+        i = int(t) // 64
+        sel = mask[0, i * (i + 1) // 2: i * (i + 1) // 2 + i + 1]
+        keys = sum(min(64, int(t) - 64 * int(j) + 1) for j in np.nonzero(sel)[0])
+        flops += 4 * keys * 128
+    return {"value": round(dec_gbs, 4), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
+            "sample": "decode: anchor top-k + %d layers for %d of %d sequences (all %d heads), %.1f s; "
+                      "prefill: RBS selection for 1 head + 256 sampled query rows, %.1f s"
+                      % (c["layers"], nseq, c["B"], c["Hq"], t_dec, t_pre),
+            "prefill_tflops": round(flops / t_pre / 1e12, 6), "seconds": round(t_dec + t_pre, 2)}
+
+
+def reference_arm(args):
+    """The reference arm is the CPU oracle: each step runs the bounded sample
+    on the host cores, rank 0 only."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import torch
+    cfg = Cfg(small=args.small)
+    dev = torch.device("cuda", 0) if torch.cuda.is_available() else torch.device("cpu")
+    # the oracle needs no GPU; the workload is generated with the same seeds
+    from sparse_attention_aware_b200 import workloads as W
+    c = cfg.dec
+    dec = W.gqa_decode(1005, device="cpu", B=4, Hq=c["Hq"], Hkv=c["Hkv"], d=c["d"], L=c["L"], P=c["P"],
+                       k=c["k"], layers=c["layers"], num_splits=c["splits"])
+    p = cfg.pre
+    pre = W.clustered_prefill(1005, device="cpu", T=p["T"], Hq=2, Hkv=1, d=p["d"], block=p["block"])
+    pc, pr = 0.95, 0.97
+    samples = []
+    t0 = time.time()
+    for _ in range(args.steps):
+        samples.append(cpu_baseline(cfg, dec, pre, pc, pr, budget_s=5.0))
+    wall = time.time() - t0
+    v = statistics.mean(s["value"] for s in samples)
+    res = {"impl": "reference", "metric": METRIC, "value": round(v, 4), "unit": "GB/s", "n_gpus": world,
+           "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(1e3 * wall / max(args.steps, 1), 1),
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+           "data": "synthetic (seeded)", "config": {"workload": WORKLOAD + " [oracle sample per step]"},
+           "cpu_baseline": {"kind": "oracle", "cores": samples[0]["cores"], "sample": samples[0]["sample"],
+                            "value": round(v, 4), "unit": "GB/s"},
+           "e2e": {"value": round(v, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(res))
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main() or 0)
