@@ -234,6 +234,45 @@ SA_API sa_status sa_sparse_decode_attn(const sa_kv_cache *kv, const void *q, sa_
                                 size_t ws_bytes, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* 3b. sa_sparse_decode_attn_noalloc -- decode without a caller workspace   */
+/* ------------------------------------------------------------------------ */
+/*
+ * The pages have no counterpart to this entry point.  It is for callers that
+ * are not able to allocate device memory: for example a plugin that its host
+ * engine hands only input and output buffers (the engine owns every device
+ * allocation), or a latency-critical serving loop that must never call into
+ * an allocator.  Such callers cannot provide the workspace that
+ * sa_sparse_decode_attn needs for its split-KV partial states.
+ *
+ * It computes exactly what sa_sparse_decode_attn computes (same kernels, same
+ * arguments except the workspace, bitwise the same results) and allocates
+ * nothing: its scratch is a device array of SA_NOALLOC_DECODE_SCRATCH_BYTES
+ * (8 MiB) built into libsa, which every GPU that loads the library holds
+ * until the process exits.
+ *   Limit: 256 + round_up_256(batch*num_q_heads*num_splits*head_dim*4)
+ *          + round_up_256(batch*num_q_heads*num_splits*8) must not exceed
+ *          8 MiB; larger calls return SA_ERR_UNSUPPORTED with nothing enqueued.
+ *   Set-up: the first call on each device looks up the array's device address
+ *          (with that device current); make that first call before any stream
+ *          capture begins.
+ *   Sharing: every call on a device uses the same array, which keeps the last
+ *          call's contents.  Calls whose GPU work overlaps in time (different
+ *          streams, or threads without ordering) race on it and corrupt each
+ *          other's results; order them.  Nothing in it needs to start zeroed:
+ *          each call rewrites every partial state it reads.
+ *   Errors: the same host-side checks as sa_sparse_decode_attn.  Bad device
+ *          data is still skipped by the kernels, but its record stays inside
+ *          the library's array and is not reported; use sa_sparse_decode_attn
+ *          with a workspace when those checks must be read.
+ */
+#define SA_NOALLOC_DECODE_SCRATCH_BYTES (8u * 1024u * 1024u)
+
+SA_API sa_status sa_sparse_decode_attn_noalloc(const sa_kv_cache *kv, const void *q, sa_dtype q_dtype,
+                                               int32_t num_q_heads, const sa_selection *sel,
+                                               float scale, int32_t num_splits, void *out,
+                                               float *lse_out, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* 4. sa_sparse_prefill_attn -- causal block-sparse prefill (tcgen05)       */
 /* ------------------------------------------------------------------------ */
 /*

@@ -1,0 +1,81 @@
+// sa_sparse_decode_attn_noalloc: split-KV sparse decode for callers that
+// cannot allocate device memory.
+//
+// Its scratch (the split-KV partial states and a status header) lives in a
+// file-scope device array of fixed size, compiled into the library.  Host code
+// never passes the array's name to a kernel (in host code it only stands in
+// for the symbol); the device address is looked up once per device with
+// cudaGetSymbolAddress and handed to the same decode kernels the workspace
+// entry point launches.
+#include <cuda_runtime.h>
+#include <mutex>
+
+#include "sa.h"
+#include "sa_internal.h"
+
+using namespace sa;
+
+namespace {
+
+constexpr size_t kNoAllocBytes = SA_NOALLOC_DECODE_SCRATCH_BYTES;
+constexpr size_t kHead = 256;   // status header, as in a workspace
+constexpr int kMaxDevices = 128;
+
+// Every GPU that loads libsa holds this array until the process exits.
+static __device__ __align__(256) unsigned char g_decode_scratch[kNoAllocBytes];
+
+std::mutex g_mu;
+void *g_scratch_ptr[kMaxDevices] = {};
+
+// Device address of g_decode_scratch on the current device (set up on the
+// first call per device).
+sa_status scratch_address(void **out)
+{
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+        cudaGetLastError();
+        return SA_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_scratch_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
+            cudaGetLastError();
+            return SA_ERR_CUDA;
+        }
+        g_scratch_ptr[dev] = p;
+    }
+    *out = g_scratch_ptr[dev];
+    return SA_OK;
+}
+
+inline size_t round_up(size_t x) { return (x + 255) / 256 * 256; }
+
+}  // namespace
+
+extern "C" sa_status sa_sparse_decode_attn_noalloc(const sa_kv_cache *kv, const void *q, sa_dtype q_dtype,
+                                                   int32_t num_q_heads, const sa_selection *sel, float scale,
+                                                   int32_t num_splits, void *out, float *lse_out,
+                                                   sa_stream_t stream)
+{
+    // argument checks: identical rules to sa_sparse_decode_attn, run first
+    if (!kv || !sel) return SA_ERR_INVALID_ARGUMENT;
+    if (kv->batch < 0 || kv->num_kv_heads <= 0 || kv->head_dim <= 0 || kv->page_size <= 0 ||
+        kv->max_pages_per_seq < 0 || kv->num_pages < 0)
+        return SA_ERR_INVALID_ARGUMENT;
+    if (kv->head_dim != 64 && kv->head_dim != 128) return SA_ERR_UNSUPPORTED;
+    if (kv->page_size != 16 && kv->page_size != 64) return SA_ERR_UNSUPPORTED;
+    if (num_q_heads <= 0 || num_splits < 1 || num_splits > 64) return SA_ERR_INVALID_ARGUMENT;
+    if (num_q_heads % kv->num_kv_heads) return SA_ERR_UNSUPPORTED;
+    const size_t rows = (size_t)kv->batch * num_q_heads;
+    const size_t need = kHead + round_up(rows * num_splits * kv->head_dim * sizeof(float)) +
+                        round_up(rows * num_splits * 2 * sizeof(float));
+    if (need > kNoAllocBytes) return SA_ERR_UNSUPPORTED;   // beyond the built-in scratch
+    void *base = nullptr;
+    sa_status st = scratch_address(&base);
+    if (st != SA_OK) return st;
+    // the workspace entry point does the remaining checks and the launches,
+    // with the static scratch standing in for the caller's workspace
+    return sa_sparse_decode_attn(kv, q, q_dtype, num_q_heads, sel, scale, num_splits, out, lse_out, base,
+                                 kNoAllocBytes, stream);
+}
