@@ -303,9 +303,10 @@ def main():
     step = Step(cfg, dec, pre, msk, pc, pr, dev)
     # selected tiles / executed (super-block union) tiles of the prefill
     csr = step.rbs_select(pre.q)
+    step.prefill(pre.q, csr)
     torch.cuda.synchronize()
     sel_tiles = int(csr.row_ptr[-1])
-    exec_tiles = union_tiles(csr, pre.q.shape[1], step.nB)
+    exec_tiles = 2 * union_tiles(csr, pre.q.shape[1], step.nB, step.ws[3])
 
     stream = torch.cuda.current_stream()
     ev = lambda: torch.cuda.Event(enable_timing=True)
@@ -403,7 +404,9 @@ def main():
                    "tokens_per_s": round(world * K * cfg.dec["B"] / (dec_ms * 1e-3), 1)},
         "prefill": {"tflops": round(pre_tflops, 2), "frac_bf16_sustained": round(per_gpu_pre / pk["bf16_tflops_sustained"], 4),
                     "frac_bf16_burst": round(per_gpu_pre / pk["bf16_tflops"], 4),
-                    "ms": round(pre_ms / K, 4), "selected_tiles": sel_tiles, "executed_tiles": exec_tiles,
+                    "ms": round(pre_ms / K, 4), "selected_tiles": sel_tiles,
+                    "executed_tiles_64x64": exec_tiles,
+                    "executed_tflops": round(world * K * exec_tiles * TILE_FLOPS / (pre_ms * 1e-3) / 1e12, 2),
                     "tokens_per_s": round(world * K * T / (pre_ms * 1e-3), 1)},
         "rbs_select": {"ms": round(rbs_ms / K, 4), "gbs": round(world * K * rbs_bytes / (rbs_ms * 1e-3) / 1e9, 2),
                        "frac_hbm": round(K * rbs_bytes / (rbs_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
@@ -451,22 +454,28 @@ def load_traffic():
         return None
 
 
-def union_tiles(csr, Hq, nB):
-    """Key tiles the prefill kernel executes: per 128-row super-block, the
-    union of its two CSR rows."""
+def union_tiles(csr, Hq, nB, ws):
+    """Key tiles the prefill kernel executes: per work item (two 64-row halves
+    read from the schedule the last prefill call left in its workspace), the
+    union of the halves' CSR rows."""
     import numpy as np
+    import torch
     rp = csr.row_ptr.cpu().numpy().astype(np.int64)
     cols = csr.cols[: int(rp[-1])].cpu().numpy()
+    buf = ws.buf
+    off = (-buf.data_ptr()) % 256 + 256
+    n_items = (buf.numel() - off) // 16
+    items = buf[off: off + 16 * n_items].view(torch.int32).reshape(-1, 4).cpu().numpy()
     tot = 0
-    for h in range(Hq):
-        for I in range((nB + 1) // 2):
-            r0 = h * nB + 2 * I
-            a = cols[rp[r0]:rp[r0 + 1]]
-            if 2 * I + 1 < nB:
-                b = cols[rp[r0 + 1]:rp[r0 + 2]]
-                tot += len(np.union1d(a, b))
-            else:
-                tot += len(a)
+    for h0, i0, h1, i1 in items:
+        if h0 < 0 or h0 >= Hq or i0 < 0 or i0 >= nB:
+            continue
+        a = cols[rp[h0 * nB + i0]:rp[h0 * nB + i0 + 1]]
+        if 0 <= h1 < Hq and 0 <= i1 < nB:
+            b = cols[rp[h1 * nB + i1]:rp[h1 * nB + i1 + 1]]
+            tot += len(np.union1d(a, b))
+        else:
+            tot += len(a)
     return int(tot)
 
 

@@ -5,25 +5,31 @@
 // item 2): for query block i of head h, attend only to the key blocks of CSR
 // row (h, i), causal inside the diagonal block, exact softmax over them.
 //
-// B200 design (one CTA = 128 query rows = query blocks 2I and 2I+1 of one
-// head, over the union of their two CSR rows; 192 threads, 2 CTAs per SM):
-//   warp 0      TMA producer: Q tile once (3-D map over [T][Hq][128]), then per
-//               selected key block the K and V page tiles (2-D maps over the
-//               paged cache; page table resolved per block), 128-byte swizzle,
-//               into an NS-stage ring guarded by mbarriers.
+// B200 design.  tcgen05 MMAs run at full rate with M = 128 rows, while a
+// query block has 64.  One CTA therefore serves a work item of two 64-row
+// halves that share their K/V tiles: two query heads of one GQA group at the
+// same query block (the pairing is chosen per block by k_prefill_schedule,
+// greedily by the overlap of their CSR rows), or, for odd group sizes, two
+// adjacent query blocks of one head.  The CTA walks the union of the two rows;
+// a key block listed by one half only is masked (p = 0) for the other half.
+//   warp 0      TMA producer: the Q halves (3-D map over [T][Hq][128]), then
+//               per key block of the merged list the K and V page tiles (2-D
+//               maps over the paged cache; page table resolved per block),
+//               128-byte swizzle, NS-stage ring.  It alone merges the two CSR
+//               rows and posts (block, half mask) in a shared-memory slot per
+//               stage, with an end sentinel.
 //   warp 1      MMA issuer (one thread) and TMEM owner: S = Q K^T (M=128, N=64,
 //               K=128) into one of two TMEM S buffers, then O += P V (M=128,
-//               N=128, K=64) into the TMEM O accumulator, in the order
-//               S_0, S_1, PV_0, S_2, PV_1, ... so the next scores are computed
-//               while the softmax of the current block runs.
-//   warps 2-5   softmax: one query row per thread (TMEM lane), row-half
-//               selection mask and causal mask, online softmax in the base-2
-//               domain with lazy rescaling (O and l are rescaled only when
-//               the running max grows by more than 2^8), P written to shared
-//               memory as bf16 in the swizzled K-major layout the next MMA
-//               reads; final O / l -> bf16 and LSE.
-// The two rows of a super-block share each K/V tile; a block listed by only
-// one row is masked (p = 0) for the other row's queries.
+//               N=128, K=64) into the TMEM O accumulator, ordered S_0, S_1,
+//               PV_0, S_2, PV_1, ... so scores of the next block are computed
+//               while the softmax of the current one runs.
+//   warps 2-5   softmax: one query row per thread (TMEM lane); half-selection
+//               and causal masks (only the diagonal block needs per-element
+//               masking); base-2 online softmax with the scale folded into the
+//               exponent's FMA and lazy rescaling (O and l rescaled only when
+//               the running max grows by more than 2^8); P written to shared
+//               memory as bf16 in the swizzled K-major layout the PV MMA reads;
+//               final O / l -> bf16 and LSE.
 // Every wait is bounded (globaltimer deadline, shared abort flag): on expiry
 // the kernel records SA_ERR_TIMEOUT, drains its own outstanding copies and
 // MMAs with bounded waits, frees its TMEM and returns.
@@ -33,6 +39,18 @@
 #include "tc_ptx.cuh"
 
 namespace sa {
+
+namespace {
+constexpr int kMaxPairGroup = 16;   // GQA groups up to 16 heads are head-paired
+}
+
+int prefill_items(int Hq, int Hkv, int nQB)
+{
+    const int G = Hq / Hkv;
+    if (G % 2 == 0 && G <= kMaxPairGroup) return (Hq / 2) * nQB;
+    return Hq * ((nQB + 1) / 2);
+}
+
 namespace {
 
 using namespace tc;
@@ -42,7 +60,7 @@ constexpr int kTmemCols = 256;                 // S0 [0,64) S1 [64,128) O [128,2
 constexpr uint32_t kQBytes = 128 * 128 * 2;     // 32 KB
 constexpr uint32_t kKVBytes = 64 * 128 * 2;     // 16 KB per K (or V) block
 constexpr uint32_t kPBytes = 128 * 64 * 2;      // 16 KB
-constexpr uint64_t kWaitNs = 400ull * 1000 * 1000;   // 0.4 s per wait
+constexpr uint64_t kWaitNs = 400ull * 1000 * 1000;   // 0.4 s
 
 constexpr uint32_t IDESC_S = idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, 0, 1);
@@ -56,77 +74,56 @@ struct Smem {
     static constexpr uint32_t BAR = P + kPBytes;
     // barriers: q_full, kfull[NS], vfull[NS], kv_empty[NS], s_full[2], s_empty[2], p_full, pv_done
     static constexpr int NBAR = 1 + 3 * NS + 6;
-    static constexpr uint32_t MISC = BAR + NBAR * 8;
+    static constexpr uint32_t SLOT = BAR + NBAR * 8;       // int2 slot[NS]
+    static constexpr uint32_t MISC = SLOT + NS * 8;
     static constexpr uint32_t TOTAL = MISC + 16;
 };
 
-// Ascending merge of the two CSR rows of a super-block; yields (key block,
-// row-half mask).  Entries out of [0, i] or not strictly ascending are
-// recorded as a fault and skipped (identically by every role).
+// Valid extent of CSR row `row` (entries <= lim): its first column pointer
+// and length, clamped to the cols capacity; malformed rows are recorded and
+// read as empty.
+__device__ __forceinline__ int csr_row(const PrefillArgs &a, int row, int lim, const int32_t *&ptr)
+{
+    const int b = __ldg(a.row_ptr + row), e = __ldg(a.row_ptr + row + 1);
+    int n = e - b;
+    ptr = a.cols + (b > 0 ? b : 0);
+    if (b < 0 || n < 0 || n > lim + 1) {
+        fault(a.st, CHK_CSR, row);
+        return 0;
+    }
+    if ((long long)b + n > a.nnz_cap) {
+        fault(a.st, CHK_CSR, row);
+        n = (long long)b >= a.nnz_cap ? 0 : (int)(a.nnz_cap - b);
+    }
+    return n;
+}
+
+// Ascending merge of the two rows of a work item -> (key block, half mask).
+// Entries out of [0, lim] or not strictly ascending are recorded and skipped.
 struct Merge {
-    const int32_t *c0, *c1;
-    int n0, n1, i0, i1, lim0, lim1, last0, last1;
+    const int32_t *c[2];
+    int n[2], i[2], lim[2], last[2];
     DevStatus *st;
 
-    __device__ void init(const PrefillArgs &a, int r0, int lim_0, bool has1)
+    __device__ int head(int h)
     {
-        st = a.st;
-        // rows are read only inside [0, nnz_cap): a truncated (overflowed) CSR
-        // loses its tail entries, it never reads past the cols buffer
-        const int b0 = __ldg(a.row_ptr + r0), e0 = __ldg(a.row_ptr + r0 + 1);
-        c0 = a.cols + (b0 > 0 ? b0 : 0);
-        n0 = e0 - b0;
-        if (b0 < 0 || n0 < 0 || n0 > lim_0 + 1) {
-            fault(st, CHK_CSR, r0);
-            n0 = 0;
-        } else if ((long long)b0 + n0 > a.nnz_cap) {
-            fault(st, CHK_CSR, r0);
-            n0 = (long long)b0 >= a.nnz_cap ? 0 : (int)(a.nnz_cap - b0);
+        while (i[h] < n[h]) {
+            const int v = __ldg(c[h] + i[h]);
+            if (v > last[h] && v <= lim[h]) return v;
+            fault(st, CHK_CSR, v);
+            ++i[h];
         }
-        n1 = 0;
-        c1 = c0;
-        if (has1) {
-            const int b1 = __ldg(a.row_ptr + r0 + 1), e1 = __ldg(a.row_ptr + r0 + 2);
-            c1 = a.cols + (b1 > 0 ? b1 : 0);
-            n1 = e1 - b1;
-            if (b1 < 0 || n1 < 0 || n1 > lim_0 + 2) {
-                fault(st, CHK_CSR, r0 + 1);
-                n1 = 0;
-            } else if ((long long)b1 + n1 > a.nnz_cap) {
-                fault(st, CHK_CSR, r0 + 1);
-                n1 = (long long)b1 >= a.nnz_cap ? 0 : (int)(a.nnz_cap - b1);
-            }
-        }
-        i0 = i1 = 0;
-        lim0 = lim_0;
-        lim1 = lim_0 + 1;
-        last0 = last1 = -1;
+        return INT_MAX;
     }
 
     __device__ bool next(int &j, int &m)
     {
-        int v0 = INT_MAX, v1 = INT_MAX;
-        while (i0 < n0) {
-            v0 = __ldg(c0 + i0);
-            if (v0 > last0 && v0 <= lim0) break;
-            fault(st, CHK_CSR, v0);
-            v0 = INT_MAX;
-            ++i0;
-        }
-        while (i1 < n1) {
-            v1 = __ldg(c1 + i1);
-            if (v1 > last1 && v1 <= lim1) break;
-            fault(st, CHK_CSR, v1);
-            v1 = INT_MAX;
-            ++i1;
-        }
-        if (i0 >= n0) v0 = INT_MAX;
-        if (i1 >= n1) v1 = INT_MAX;
+        const int v0 = head(0), v1 = head(1);
         if (v0 == INT_MAX && v1 == INT_MAX) return false;
         j = min(v0, v1);
         m = (v0 == j ? 1 : 0) | (v1 == j ? 2 : 0);
-        if (v0 == j) { last0 = v0; ++i0; }
-        if (v1 == j) { last1 = v1; ++i1; }
+        if (v0 == j) { last[0] = v0; ++i[0]; }
+        if (v1 == j) { last[1] = v1; ++i[1]; }
         return true;
     }
 };
@@ -152,16 +149,17 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t *s_empty = s_full + 2;
     uint64_t *p_full = s_empty + 2;
     uint64_t *pv_done = p_full + 1;
+    volatile int *slots = reinterpret_cast<volatile int *>(smem + L::SLOT);   // (j, mask) per stage
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC + 4);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int nQB = (a.T + 63) >> 6, nSB = (nQB + 1) >> 1;
-    const int I = nSB - 1 - (int)(blockIdx.x / a.Hq);   // heavy (late) rows first
-    const int h = (int)(blockIdx.x % a.Hq);
-    const int g = h / (a.Hq / a.c.Hkv);
-    const int r0 = h * nQB + 2 * I;
-    const bool has1 = 2 * I + 1 < nQB;
+    const int nQB = (a.T + 63) >> 6;
+    const int4 item = a.items[blockIdx.x];
+    const bool has_b = item.z >= 0;
+    const int hq[2] = {item.x, has_b ? item.z : item.x};
+    const int iq[2] = {item.y, has_b ? item.w : item.y};
+    const int g = hq[0] / (a.Hq / a.c.Hkv);
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
@@ -186,9 +184,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t tmem = *tmem_slot;
     const uint64_t deadline = globaltimer() + kWaitNs * 4;
 
-    Merge mg;
-    mg.init(a, r0, 2 * I, has1);
-
     if (warp == 0) {
         // ------------------------------------------------------------ producer
         if (lane == 0) {
@@ -196,19 +191,40 @@ __global__ void __launch_bounds__(kThreads, 2)
             prefetch_tmap(&tmK);
             prefetch_tmap(&tmV);
             mbar_arrive_expect_tx(q_full, kQBytes);
-            tma_load_3d(smem + L::Q, &tmQ, q_full, 0, h, 128 * I);
-            tma_load_3d(smem + L::Q + kQBytes / 2, &tmQ, q_full, 64, h, 128 * I);
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+                for (int c = 0; c < 2; ++c)
+                    tma_load_3d(smem + L::Q + c * (kQBytes / 2) + hf * (kQBytes / 4), &tmQ, q_full, 64 * c, hq[hf],
+                                64 * iq[hf]);
+            Merge mg;
+            mg.st = a.st;
+            mg.n[0] = csr_row(a, hq[0] * nQB + iq[0], iq[0], mg.c[0]);
+            mg.n[1] = has_b ? csr_row(a, hq[1] * nQB + iq[1], iq[1], mg.c[1]) : 0;
+            if (!has_b) mg.c[1] = mg.c[0];
+            mg.i[0] = mg.i[1] = 0;
+            mg.lim[0] = iq[0];
+            mg.lim[1] = iq[1];
+            mg.last[0] = mg.last[1] = -1;
             int n = 0, j, m;
             bool ok = true;
-            while (ok && mg.next(j, m)) {
+            for (;;) {
                 const int s = n % NS;
                 if (n >= NS) ok = mbar_wait(kv_empty + s, ((n / NS) - 1) & 1, deadline, abort_flag);
                 if (!ok) break;
+                if (!mg.next(j, m)) {
+                    slots[2 * s] = -1;                 // end of the list
+                    slots[2 * s + 1] = 0;
+                    mbar_arrive(kfull + s);
+                    break;
+                }
                 int page = __ldg(a.c.pt + j);
                 if (page < 0 || page >= a.c.num_pages) {
                     fault(a.st, CHK_PAGE, page);
                     page = 0;
                 }
+                slots[2 * s] = j;
+                slots[2 * s + 1] = m;
                 const int row = (page * a.c.Hkv + g) * 64;
                 uint8_t *kd = smem + L::K + s * kKVBytes;
                 uint8_t *vd = smem + L::V + s * kKVBytes;
@@ -223,10 +239,7 @@ __global__ void __launch_bounds__(kThreads, 2)
             if (!ok) {
                 *abort_flag = 1;
                 record(a.st, SA_ERR_TIMEOUT, CHK_WAIT, 0);
-            }
-            // never leave with copies in flight: the last NS loads are consumed
-            // by the MMA thread in the normal case; on abort wait for them here
-            if (*abort_flag) {
+                // never leave with copies in flight
                 const uint64_t dl2 = globaltimer() + kWaitNs;
                 volatile int never = 0;
                 for (int p = max(0, n - NS); p < n; ++p) {
@@ -239,7 +252,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // ------------------------------------------------------------ MMA
         if (lane == 0) {
             const uint32_t qa = sbase + L::Q;
-            int n = 0, j, m;
+            int n = 0;
             bool ok = mbar_wait(q_full, 0, deadline, abort_flag);
             auto issue_pv = [&](int p) -> bool {
                 const int sp = p % NS;
@@ -258,10 +271,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                 mma_commit(kv_empty + sp);
                 return true;
             };
-            while (ok && mg.next(j, m)) {
+            while (ok) {
                 const int s = n % NS;
                 ok = mbar_wait(kfull + s, (n / NS) & 1, deadline, abort_flag);
-                if (ok && n >= 2) ok = mbar_wait(s_empty + (n & 1), ((n - 2) >> 1) & 1, deadline, abort_flag);
+                if (!ok || slots[2 * s] < 0) break;
+                if (n >= 2) ok = mbar_wait(s_empty + (n & 1), ((n - 2) >> 1) & 1, deadline, abort_flag);
                 if (!ok) break;
                 fence_after_sync();
                 const uint32_t ka = sbase + L::K + s * kKVBytes;
@@ -285,61 +299,78 @@ __global__ void __launch_bounds__(kThreads, 2)
         // ------------------------------------------------------------ softmax
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
-        const int qpos = 128 * I + r;
-        const int half = r >> 6;
+        const int hf = r >> 6;                       // warp-uniform half
+        const int rr = r & 63;
+        const int qpos = 64 * iq[hf] + rr;
         const uint32_t lane_base = tmem + ((uint32_t)(32 * q4) << 16);
-        const float C = a.scale * kLog2e;
+        const float C = a.scale * kLog2e;            // > 0 (checked on the host)
         float m_used = -INFINITY, l = 0.f;
-        int n = 0, j, msk;
+        int n = 0;
         bool ok = true;
         uint8_t *prow = smem + L::P + r * 128;
-        while (ok && mg.next(j, msk)) {
+        for (;;) {
+            const int s = n % NS;
+            ok = __all_sync(0xffffffffu, mbar_wait(kfull + s, (n / NS) & 1, deadline, abort_flag));
+            if (!ok) break;
+            const int2 sl = make_int2(slots[2 * s], slots[2 * s + 1]);
+            if (sl.x < 0) break;
             ok = __all_sync(0xffffffffu, mbar_wait(s_full + (n & 1), (n >> 1) & 1, deadline, abort_flag));
             if (!ok) break;
             fence_after_sync();
-            uint32_t sr[64];
-            tmem_ld32(lane_base + (n & 1) * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
-            tmem_ld32(lane_base + (n & 1) * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
-            tmem_wait_ld();
-            fence_before_sync();
-            mbar_arrive(s_empty + (n & 1));
-
-            const bool sel = (msk >> half) & 1;
-            const int kb = 64 * j;
-            const int lim = qpos - kb;   // key offsets c <= lim are causal-valid
-            float v[64];
-            float rowmax = -INFINITY;
-#pragma unroll
-            for (int c = 0; c < 64; ++c) {
-                const bool valid = sel && (c <= lim);
-                const float x = valid ? __uint_as_float(sr[c]) * C : -INFINITY;
-                v[c] = x;
-                rowmax = fmaxf(rowmax, x);
-            }
-            const float m_new = fmaxf(m_used, rowmax);
-            bool rescale = false;
-            float alpha = 1.f;
-            if (m_new > -INFINITY) {
-                if (m_used == -INFINITY) {
-                    m_used = m_new;
-                } else if (m_new > m_used + 8.f) {
-                    alpha = ex2(m_used - m_new);
-                    l *= alpha;
-                    m_used = m_new;
-                    rescale = true;
-                }
-            }
-            const float base = (m_used == -INFINITY) ? 0.f : m_used;
+            const bool sel = (sl.y >> hf) & 1;       // warp-uniform
             uint32_t pk[32];
-            float psum = 0.f;
+            float alpha = 1.f;
+            bool rescale = false;
+            if (sel) {
+                uint32_t sr[64];
+                tmem_ld32(lane_base + (n & 1) * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
+                tmem_ld32(lane_base + (n & 1) * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
+                tmem_wait_ld();
+                fence_before_sync();
+                mbar_arrive(s_empty + (n & 1));
+                float v[64];
+                float mx = -INFINITY;
+                if (sl.x == iq[hf]) {                // diagonal block: causal inside
 #pragma unroll
-            for (int c = 0; c < 64; c += 2) {
-                const float p0 = ex2(v[c] - base);
-                const float p1 = ex2(v[c + 1] - base);
-                psum += p0 + p1;
-                pk[c >> 1] = pack_bf16x2(p0, p1);
+                    for (int c = 0; c < 64; ++c) {
+                        v[c] = c <= rr ? __uint_as_float(sr[c]) : -INFINITY;
+                        mx = fmaxf(mx, v[c]);
+                    }
+                } else {
+#pragma unroll
+                    for (int c = 0; c < 64; ++c) {
+                        v[c] = __uint_as_float(sr[c]);
+                        mx = fmaxf(mx, v[c]);
+                    }
+                }
+                const float m_new = fmaxf(m_used, mx * C);
+                if (m_new > -INFINITY) {
+                    if (m_used == -INFINITY) {
+                        m_used = m_new;
+                    } else if (m_new > m_used + 8.f) {
+                        alpha = ex2(m_used - m_new);
+                        l *= alpha;
+                        m_used = m_new;
+                        rescale = true;
+                    }
+                }
+                const float nb = (m_used == -INFINITY) ? 0.f : -m_used;
+                float ps0 = 0.f, ps1 = 0.f;
+#pragma unroll
+                for (int c = 0; c < 64; c += 2) {
+                    const float p0 = ex2(fmaf(v[c], C, nb));
+                    const float p1 = ex2(fmaf(v[c + 1], C, nb));
+                    ps0 += p0;
+                    ps1 += p1;
+                    pk[c >> 1] = pack_bf16x2(p0, p1);
+                }
+                l += ps0 + ps1;
+            } else {
+                fence_before_sync();
+                mbar_arrive(s_empty + (n & 1));
+#pragma unroll
+                for (int c = 0; c < 32; ++c) pk[c] = 0u;
             }
-            l += psum;
             if (n > 0) {
                 ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (n - 1) & 1, deadline, abort_flag));
                 if (!ok) break;
@@ -376,10 +407,11 @@ __global__ void __launch_bounds__(kThreads, 2)
             *abort_flag = 1;
             record(a.st, SA_ERR_TIMEOUT, CHK_WAIT, 2);
         }
-        // epilogue: O / l -> bf16, LSE
-        const bool store = qpos < a.T && ok;
+        // epilogue: O / l -> bf16, LSE (the second half of a one-row item is
+        // never stored)
+        const bool store = qpos < a.T && ok && (hf == 0 || has_b);
         const float inv = l > 0.f ? 1.f / l : 0.f;
-        uint16_t *orow = a.out + ((size_t)qpos * a.Hq + h) * 128;
+        uint16_t *orow = a.out + ((size_t)qpos * a.Hq + hq[hf]) * 128;
 #pragma unroll 1
         for (int c4 = 0; c4 < 4; ++c4) {
             uint32_t o[32];
@@ -402,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
             }
         }
-        if (store && a.lse) a.lse[(size_t)qpos * a.Hq + h] = l > 0.f ? (m_used + lg2(l)) * kLn2 : -INFINITY;
+        if (store && a.lse) a.lse[(size_t)qpos * a.Hq + hq[hf]] = l > 0.f ? (m_used + lg2(l)) * kLn2 : -INFINITY;
         fence_before_sync();
     }
 
@@ -411,13 +443,12 @@ __global__ void __launch_bounds__(kThreads, 2)
         fence_after_sync();
         if (*abort_flag) {
             // bounded drain of outstanding MMAs before TMEM is freed: a fresh
-            // commit on the (otherwise idle) pv_done barrier arrives once every
-            // earlier tcgen05 op of the issuing thread has completed
+            // commit on pv_done arrives once every earlier tcgen05 op of the
+            // issuing thread has completed
             if (lane == 0) {
                 volatile int never = 0;
                 const uint64_t dl = globaltimer() + kWaitNs;
                 mma_commit(pv_done);
-                // either phase may be the drain's; wait for both parities in turn
                 mbar_wait(pv_done, 0, dl, &never);
                 mbar_wait(pv_done, 1, dl, &never);
             }
@@ -425,6 +456,76 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
         tmem_dealloc(tmem, kTmemCols);
     }
+}
+
+// ---------------------------------------------------------------------------
+// Work items.  Even GQA group sizes (<= 16): per (kv head g, query block i),
+// pair the group's query heads greedily by the waste of their union (|A| +
+// |B| - 2|A n B|, smallest first, ties to the lowest pair).  One warp per
+// (g, i).  Items are ordered by query block, latest first (heavier rows early).
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_prefill_schedule_pairs(const PrefillArgs a)
+{
+    __shared__ int cost[8][kMaxPairGroup][kMaxPairGroup];
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int nQB = (a.T + 63) >> 6;
+    const int G = a.Hq / a.c.Hkv;
+    const int task = blockIdx.x * 8 + warp;
+    if (task >= a.c.Hkv * nQB) return;
+    const int g = task / nQB, i = task % nQB;
+    const int npairs = G * (G - 1) / 2;
+    for (int p = lane; p < npairs; p += 32) {
+        int x = 0, pa = 0, pb = 1;
+        for (pa = 0; pa < G - 1; ++pa) {
+            if (p < x + (G - 1 - pa)) {
+                pb = pa + 1 + (p - x);
+                break;
+            }
+            x += G - 1 - pa;
+        }
+        const int32_t *ca, *cb;
+        const int na = csr_row(a, (g * G + pa) * nQB + i, i, ca);
+        const int nb = csr_row(a, (g * G + pb) * nQB + i, i, cb);
+        int ia = 0, ib = 0, inter = 0;
+        while (ia < na && ib < nb) {
+            const int va = __ldg(ca + ia), vb = __ldg(cb + ib);
+            inter += va == vb;
+            ia += va <= vb;
+            ib += vb <= va;
+        }
+        cost[warp][pa][pb] = na + nb - 2 * inter;
+    }
+    __syncwarp();
+    if (lane == 0) {
+        unsigned used = 0;
+        const int base = (nQB - 1 - i) * (a.Hq / 2) + g * (G / 2);
+        for (int t = 0; t < G / 2; ++t) {
+            int best = INT_MAX, ba = 0, bb = 1;
+            for (int pa = 0; pa < G; ++pa) {
+                if (used >> pa & 1) continue;
+                for (int pb = pa + 1; pb < G; ++pb) {
+                    if (used >> pb & 1) continue;
+                    if (cost[warp][pa][pb] < best) {
+                        best = cost[warp][pa][pb];
+                        ba = pa;
+                        bb = pb;
+                    }
+                }
+            }
+            used |= (1u << ba) | (1u << bb);
+            a.items[base + t] = make_int4(g * G + ba, i, g * G + bb, i);
+        }
+    }
+}
+
+// Odd group sizes: adjacent query blocks (2I, 2I+1) of one head, latest first.
+__global__ void k_prefill_schedule_adjacent(const PrefillArgs a)
+{
+    const int nQB = (a.T + 63) >> 6, nSB = (nQB + 1) >> 1;
+    const int x = blockIdx.x * blockDim.x + threadIdx.x;
+    if (x >= a.Hq * nSB) return;
+    const int I = nSB - 1 - x / a.Hq, h = x % a.Hq;
+    a.items[x] = make_int4(h, 2 * I, 2 * I + 1 < nQB ? h : -1, 2 * I + 1);
 }
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
@@ -449,7 +550,7 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s)
     {
         cuuint64_t dims[3] = {128, (cuuint64_t)a.Hq, (cuuint64_t)a.T};
         cuuint64_t strides[2] = {256, (cuuint64_t)a.Hq * 256};
-        cuuint32_t box[3] = {64, 1, 128};
+        cuuint32_t box[3] = {64, 1, 64};
         cuuint32_t es[3] = {1, 1, 1};
         if (enc(&mq, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, (void *)a.q, dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -467,16 +568,20 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s)
                 CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
             return cudaErrorInvalidValue;
     }
+    const int nQB = (a.T + 63) / 64;
+    const int G = a.Hq / a.c.Hkv;
+    if (a.n_items <= 0) return cudaSuccess;
+    if (G % 2 == 0 && G <= kMaxPairGroup)
+        k_prefill_schedule_pairs<<<(a.c.Hkv * nQB + 7) / 8, 256, 0, s>>>(a);
+    else
+        k_prefill_schedule_adjacent<<<(a.n_items + 255) / 256, 256, 0, s>>>(a);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     using L = Smem<kStages>;
     const size_t smem = L::TOTAL;
-    cudaError_t e = cudaFuncSetAttribute(k_prefill_tc<kStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem);
+    e = cudaFuncSetAttribute(k_prefill_tc<kStages>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    const int nQB = (a.T + 63) / 64, nSB = (nQB + 1) / 2;
-    const long long grid = (long long)nSB * a.Hq;
-    if (grid <= 0) return cudaSuccess;
-    if (grid > 0x7fffffff) return cudaErrorInvalidValue;
-    k_prefill_tc<kStages><<<(unsigned)grid, kThreads, smem, s>>>(mq, mk, mv, a);
+    k_prefill_tc<kStages><<<(unsigned)a.n_items, kThreads, smem, s>>>(mq, mk, mv, a);
     return cudaGetLastError();
 }
 

@@ -98,7 +98,11 @@ size_t ws_blocks(const sa_kv_cache *kv, const sa_block_select_args *a)
                                           a->tau_c == nullptr, offs);
 }
 
-size_t ws_prefill() { return kHeader + kAlign; }
+size_t ws_prefill(const sa_kv_cache *kv, int Hq, int T)
+{
+    const int nQB = (T + 63) / 64;
+    return kHeader + up((size_t)prefill_items(Hq, kv->num_kv_heads, nQB) * sizeof(int4) + 16);
+}
 
 }  // namespace
 
@@ -135,7 +139,8 @@ size_t sa_workspace_bytes(sa_op op, const sa_kv_cache *kv, const sa_ws_query *q)
         return ws_decode(kv, q->num_q_heads, q->num_splits);
     case SA_OP_PREFILL:
         if (q->num_q_heads <= 0 || q->num_tokens < 0) return 0;
-        return ws_prefill();
+        if (q->num_q_heads % kv->num_kv_heads) return 0;
+        return ws_prefill(kv, q->num_q_heads, q->num_tokens);
     default:
         return 0;
     }
@@ -347,7 +352,8 @@ sa_status sa_sparse_prefill_attn(const sa_kv_cache *kv, const void *q, int32_t n
     if (csr && csr->nnz_capacity < 0) return SA_ERR_INVALID_ARGUMENT;
     if ((long long)kv->num_pages * kv->num_kv_heads * 64 >= (1LL << 31)) return SA_ERR_UNSUPPORTED;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(lse_out, 4)) return SA_ERR_INVALID_ARGUMENT;
-    st = check_ws(ws, ws_bytes, ws_prefill());
+    if (!(scale > 0.f) || scale == INFINITY) return SA_ERR_INVALID_ARGUMENT;
+    st = check_ws(ws, ws_bytes, ws_prefill(kv, num_q_heads, num_tokens));
     if (st != SA_OK) return st;
     a.q = static_cast<const uint16_t *>(q);
     a.Hq = num_q_heads;
@@ -359,7 +365,8 @@ sa_status sa_sparse_prefill_attn(const sa_kv_cache *kv, const void *q, int32_t n
     a.nnz_cap = csr->nnz_capacity;
     a.out = static_cast<uint16_t *>(out);
     a.lse = lse_out;
-    a.work_counter = reinterpret_cast<int *>(static_cast<char *>(ws) + kHeader);
+    a.items = reinterpret_cast<int4 *>(static_cast<char *>(ws) + kHeader);
+    a.n_items = prefill_items(num_q_heads, kv->num_kv_heads, (num_tokens + 63) / 64);
     a.st = static_cast<DevStatus *>(ws);
     if (num_tokens == 0) return SA_OK;
     cudaError_t e = launch_prefill(a, (cudaStream_t)stream);

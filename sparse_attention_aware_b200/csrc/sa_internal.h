@@ -111,9 +111,12 @@ struct PrefillArgs {
     int64_t nnz_cap;
     uint16_t *out;
     float *lse;
-    int *work_counter;
+    int4 *items;    // workspace: per CTA {head A, q-block A, head B (-1: none), q-block B}
+    int n_items;
     DevStatus *st;
 };
+// number of prefill work items (two 64-row halves each) for a problem
+int prefill_items(int Hq, int Hkv, int nQB);
 cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s);
 
 }  // namespace sa
