@@ -137,7 +137,8 @@ typedef struct {
  *   count_out  int32 [batch][num_q_heads] = min(k, L_b)
  *   ws         workspace of sa_workspace_bytes(SA_OP_SELECT_TOPK, ...) bytes
  * Errors: SA_ERR_INVALID_ARGUMENT (k < 1, k > 65536, null pointers),
- * SA_ERR_UNSUPPORTED, SA_ERR_WORKSPACE.
+ * SA_ERR_UNSUPPORTED (also: max_pages_per_seq * page_size > 2^19 tokens),
+ * SA_ERR_WORKSPACE.
  */
 SA_API sa_status sa_select_topk(const sa_kv_cache *kv, const void *q, sa_dtype q_dtype,
                          int32_t num_q_heads, int32_t k, int32_t *idx_out, int32_t *count_out,

@@ -12,17 +12,22 @@
 // greedily by the overlap of their CSR rows), or, for odd group sizes, two
 // adjacent query blocks of one head.  The CTA walks the union of the two rows;
 // a key block listed by one half only is masked (p = 0) for the other half.
-//   warp 0      TMA producer: the Q halves (3-D map over [T][Hq][128]), then
-//               per key block of the merged list the K and V page tiles (2-D
-//               maps over the paged cache; page table resolved per block),
-//               128-byte swizzle, NS-stage ring.  It alone merges the two CSR
-//               rows and posts (block, half mask) in a shared-memory slot per
-//               stage, with an end sentinel.
+//   warp 0      K producer: the Q halves (3-D map over [T][Hq][128]), then
+//               per key block of the merged list the K page tile (2-D map over
+//               the paged cache; page table resolved per block), 128-byte
+//               swizzle, NS-stage ring released as soon as S = QK^T of that
+//               block has completed.  It merges the two CSR rows and posts
+//               (block, half mask) per stage, with an end sentinel.
+//   warp 6      V producer: the V page tiles of the same merged list into their
+//               own NS-stage ring, released when PV of that block completes.
 //   warp 1      MMA issuer (one thread) and TMEM owner: S = Q K^T (M=128, N=64,
-//               K=128) into one of two TMEM S buffers, then O += P V (M=128,
-//               N=128, K=64) into the TMEM O accumulator, ordered S_0, S_1,
-//               PV_0, S_2, PV_1, ... so scores of the next block are computed
-//               while the softmax of the current one runs.
+//               K=128) into one of two TMEM S buffers, O += P V (M=128, N=128,
+//               K=64) into the TMEM O accumulator.  S runs up to two blocks
+//               ahead of PV (S_0 S_1 S_2 PV_0 S_3 PV_1 ...); the thread polls
+//               the readiness of the next S and the next PV so neither blocks
+//               the other.  It forwards each block's (index, half mask) to the
+//               softmax through a shared ring published by a release-arrive on
+//               the S-ready barrier.
 //   warps 2-5   softmax: one query row per thread (TMEM lane); half-selection
 //               and causal masks (only the diagonal block needs per-element
 //               masking); base-2 online softmax with the scale folded into the
@@ -55,7 +60,7 @@ namespace {
 
 using namespace tc;
 
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;
 constexpr int kTmemCols = 256;                 // S0 [0,64) S1 [64,128) O [128,256)
 constexpr uint32_t kQBytes = 128 * 128 * 2;     // 32 KB
 constexpr uint32_t kKVBytes = 64 * 128 * 2;     // 16 KB per K (or V) block
@@ -72,10 +77,11 @@ struct Smem {
     static constexpr uint32_t V = K + NS * kKVBytes;
     static constexpr uint32_t P = V + NS * kKVBytes;
     static constexpr uint32_t BAR = P + kPBytes;
-    // barriers: q_full, kfull[NS], vfull[NS], kv_empty[NS], s_full[2], s_empty[2], p_full, pv_done
-    static constexpr int NBAR = 1 + 3 * NS + 6;
-    static constexpr uint32_t SLOT = BAR + NBAR * 8;       // int2 slot[NS]
-    static constexpr uint32_t MISC = SLOT + NS * 8;
+    // q_full, kfull[NS], vfull[NS], k_empty[NS], v_empty[NS], s_full[2], s_empty[2], p_full, pv_done
+    static constexpr int NBAR = 1 + 4 * NS + 6;
+    static constexpr uint32_t SLOT = BAR + NBAR * 8;       // int2 slot[NS]: K producer -> MMA
+    static constexpr uint32_t SINFO = SLOT + NS * 8;       // int2 sinfo[4]: MMA -> softmax
+    static constexpr uint32_t MISC = SINFO + 4 * 8;
     static constexpr uint32_t TOTAL = MISC + 16;
 };
 
@@ -144,12 +150,14 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t *q_full = bars;
     uint64_t *kfull = bars + 1;
     uint64_t *vfull = kfull + NS;
-    uint64_t *kv_empty = vfull + NS;
-    uint64_t *s_full = kv_empty + NS;
+    uint64_t *k_empty = vfull + NS;
+    uint64_t *v_empty = k_empty + NS;
+    uint64_t *s_full = v_empty + NS;
     uint64_t *s_empty = s_full + 2;
     uint64_t *p_full = s_empty + 2;
     uint64_t *pv_done = p_full + 1;
-    volatile int *slots = reinterpret_cast<volatile int *>(smem + L::SLOT);   // (j, mask) per stage
+    volatile int *slots = reinterpret_cast<volatile int *>(smem + L::SLOT);   // (j, mask) per K stage
+    volatile int *sinfo = reinterpret_cast<volatile int *>(smem + L::SINFO); // (j, mask) per S, ring of 4
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + L::MISC + 4);
 
@@ -166,10 +174,11 @@ __global__ void __launch_bounds__(kThreads, 2)
         for (int s = 0; s < NS; ++s) {
             mbar_init(kfull + s, 1);
             mbar_init(vfull + s, 1);
-            mbar_init(kv_empty + s, 1);
+            mbar_init(k_empty + s, 1);
+            mbar_init(v_empty + s, 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(s_full + b, 1);
+            mbar_init(s_full + b, 2);      // S MMAs complete + block info posted
             mbar_init(s_empty + b, 128);
         }
         mbar_init(p_full, 128);
@@ -184,118 +193,148 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t tmem = *tmem_slot;
     const uint64_t deadline = globaltimer() + kWaitNs * 4;
 
-    if (warp == 0) {
-        // ------------------------------------------------------------ producer
+    auto init_merge = [&](Merge &mg) {
+        mg.st = a.st;
+        mg.n[0] = csr_row(a, hq[0] * nQB + iq[0], iq[0], mg.c[0]);
+        mg.n[1] = has_b ? csr_row(a, hq[1] * nQB + iq[1], iq[1], mg.c[1]) : 0;
+        if (!has_b) mg.c[1] = mg.c[0];
+        mg.i[0] = mg.i[1] = 0;
+        mg.lim[0] = iq[0];
+        mg.lim[1] = iq[1];
+        mg.last[0] = mg.last[1] = -1;
+    };
+    auto page_row = [&](int j) {
+        int page = __ldg(a.c.pt + j);
+        if (page < 0 || page >= a.c.num_pages) {
+            fault(a.st, CHK_PAGE, page);
+            page = 0;
+        }
+        return (page * a.c.Hkv + g) * 64;
+    };
+
+    if (warp == 0 || warp == 6) {
+        // ------------------------------------------------------ K / V producers
         if (lane == 0) {
-            prefetch_tmap(&tmQ);
-            prefetch_tmap(&tmK);
-            prefetch_tmap(&tmV);
-            mbar_arrive_expect_tx(q_full, kQBytes);
+            const bool is_k = warp == 0;
+            uint64_t *full = is_k ? kfull : vfull;
+            uint64_t *empty = is_k ? k_empty : v_empty;
+            const CUtensorMap *map = is_k ? &tmK : &tmV;
+            uint8_t *ring = smem + (is_k ? L::K : L::V);
+            prefetch_tmap(map);
+            if (is_k) {
+                prefetch_tmap(&tmQ);
+                mbar_arrive_expect_tx(q_full, kQBytes);
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf)
+                for (int hf = 0; hf < 2; ++hf)
 #pragma unroll
-                for (int c = 0; c < 2; ++c)
-                    tma_load_3d(smem + L::Q + c * (kQBytes / 2) + hf * (kQBytes / 4), &tmQ, q_full, 64 * c, hq[hf],
-                                64 * iq[hf]);
+                    for (int c = 0; c < 2; ++c)
+                        tma_load_3d(smem + L::Q + c * (kQBytes / 2) + hf * (kQBytes / 4), &tmQ, q_full, 64 * c,
+                                    hq[hf], 64 * iq[hf]);
+            }
             Merge mg;
-            mg.st = a.st;
-            mg.n[0] = csr_row(a, hq[0] * nQB + iq[0], iq[0], mg.c[0]);
-            mg.n[1] = has_b ? csr_row(a, hq[1] * nQB + iq[1], iq[1], mg.c[1]) : 0;
-            if (!has_b) mg.c[1] = mg.c[0];
-            mg.i[0] = mg.i[1] = 0;
-            mg.lim[0] = iq[0];
-            mg.lim[1] = iq[1];
-            mg.last[0] = mg.last[1] = -1;
+            init_merge(mg);
             int n = 0, j, m;
             bool ok = true;
             for (;;) {
                 const int s = n % NS;
-                if (n >= NS) ok = mbar_wait(kv_empty + s, ((n / NS) - 1) & 1, deadline, abort_flag);
+                if (n >= NS) ok = mbar_wait(empty + s, ((n / NS) - 1) & 1, deadline, abort_flag);
                 if (!ok) break;
                 if (!mg.next(j, m)) {
-                    slots[2 * s] = -1;                 // end of the list
-                    slots[2 * s + 1] = 0;
-                    mbar_arrive(kfull + s);
+                    if (is_k) {
+                        slots[2 * s] = -1;             // end of the list
+                        slots[2 * s + 1] = 0;
+                        mbar_arrive(kfull + s);
+                    }
                     break;
                 }
-                int page = __ldg(a.c.pt + j);
-                if (page < 0 || page >= a.c.num_pages) {
-                    fault(a.st, CHK_PAGE, page);
-                    page = 0;
+                const int row = page_row(j);
+                if (is_k) {
+                    slots[2 * s] = j;
+                    slots[2 * s + 1] = m;
                 }
-                slots[2 * s] = j;
-                slots[2 * s + 1] = m;
-                const int row = (page * a.c.Hkv + g) * 64;
-                uint8_t *kd = smem + L::K + s * kKVBytes;
-                uint8_t *vd = smem + L::V + s * kKVBytes;
-                mbar_arrive_expect_tx(kfull + s, kKVBytes);
-                tma_load_2d(kd, &tmK, kfull + s, 0, row);
-                tma_load_2d(kd + kKVBytes / 2, &tmK, kfull + s, 64, row);
-                mbar_arrive_expect_tx(vfull + s, kKVBytes);
-                tma_load_2d(vd, &tmV, vfull + s, 0, row);
-                tma_load_2d(vd + kKVBytes / 2, &tmV, vfull + s, 64, row);
+                uint8_t *dst = ring + s * kKVBytes;
+                mbar_arrive_expect_tx(full + s, kKVBytes);
+                tma_load_2d(dst, map, full + s, 0, row);
+                tma_load_2d(dst + kKVBytes / 2, map, full + s, 64, row);
                 ++n;
             }
             if (!ok) {
                 *abort_flag = 1;
-                record(a.st, SA_ERR_TIMEOUT, CHK_WAIT, 0);
+                record(a.st, SA_ERR_TIMEOUT, CHK_WAIT, is_k ? 0 : 3);
                 // never leave with copies in flight
                 const uint64_t dl2 = globaltimer() + kWaitNs;
                 volatile int never = 0;
-                for (int p = max(0, n - NS); p < n; ++p) {
-                    mbar_wait(kfull + p % NS, (p / NS) & 1, dl2, &never);
-                    mbar_wait(vfull + p % NS, (p / NS) & 1, dl2, &never);
-                }
+                for (int p = max(0, n - NS); p < n; ++p) mbar_wait(full + p % NS, (p / NS) & 1, dl2, &never);
             }
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
         if (lane == 0) {
             const uint32_t qa = sbase + L::Q;
-            int n = 0;
+            const uint32_t pa = sbase + L::P;
             bool ok = mbar_wait(q_full, 0, deadline, abort_flag);
-            auto issue_pv = [&](int p) -> bool {
-                const int sp = p % NS;
-                if (!mbar_wait(vfull + sp, (p / NS) & 1, deadline, abort_flag)) return false;
-                if (!mbar_wait(p_full, p & 1, deadline, abort_flag)) return false;
-                fence_after_sync();
-                const uint32_t pa = sbase + L::P;
-                const uint32_t va = sbase + L::V + sp * kKVBytes;
-#pragma unroll
-                for (int kk = 0; kk < 4; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(pa + kk * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(va + kk * 2048, 8192, 1024);
-                    mma_f16(tmem + 128, ad, bd, IDESC_PV, (p > 0 || kk > 0) ? 1u : 0u);
-                }
-                mma_commit(pv_done);
-                mma_commit(kv_empty + sp);
-                return true;
-            };
+            int ns = 0, npv = 0, total = -1;
+            uint32_t idle = 0;
             while (ok) {
-                const int s = n % NS;
-                ok = mbar_wait(kfull + s, (n / NS) & 1, deadline, abort_flag);
-                if (!ok || slots[2 * s] < 0) break;
-                if (n >= 2) ok = mbar_wait(s_empty + (n & 1), ((n - 2) >> 1) & 1, deadline, abort_flag);
-                if (!ok) break;
-                fence_after_sync();
-                const uint32_t ka = sbase + L::K + s * kKVBytes;
+                bool progressed = false;
+                // next S: K landed and its S buffer read by the softmax two blocks back
+                if (total < 0 && ns < npv + 3) {
+                    const int s = ns % NS;
+                    if (mbar_try_wait(kfull + s, (ns / NS) & 1) &&
+                        (ns < 2 || mbar_try_wait(s_empty + (ns & 1), ((ns - 2) >> 1) & 1))) {
+                        const int j = slots[2 * s], m = slots[2 * s + 1];
+                        sinfo[2 * (ns & 3)] = j;
+                        sinfo[2 * (ns & 3) + 1] = m;
+                        if (j < 0) {
+                            total = ns;
+                            mbar_arrive(s_full + (ns & 1));
+                            mbar_arrive(s_full + (ns & 1));
+                        } else {
+                            fence_after_sync();
+                            const uint32_t ka = sbase + L::K + s * kKVBytes;
 #pragma unroll
-                for (int kk = 0; kk < 8; ++kk) {
-                    const uint64_t ad = smem_desc_sw128(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
-                    const uint64_t bd = smem_desc_sw128(ka + (kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32, 16, 1024);
-                    mma_f16(tmem + (n & 1) * 64, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const uint64_t ad =
+                                    smem_desc_sw128(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
+                                const uint64_t bd =
+                                    smem_desc_sw128(ka + (kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32, 16, 1024);
+                                mma_f16(tmem + (ns & 1) * 64, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+                            }
+                            mma_commit(s_full + (ns & 1));
+                            mma_commit(k_empty + s);
+                            mbar_arrive(s_full + (ns & 1));   // publishes sinfo (release)
+                            ++ns;
+                        }
+                        progressed = true;
+                    }
                 }
-                mma_commit(s_full + (n & 1));
-                if (n >= 1) ok = issue_pv(n - 1);
-                ++n;
+                // next PV: V landed and P written
+                if (npv < ns) {
+                    const int sp = npv % NS;
+                    if (mbar_try_wait(vfull + sp, (npv / NS) & 1) && mbar_try_wait(p_full, npv & 1)) {
+                        fence_after_sync();
+                        const uint32_t va = sbase + L::V + sp * kKVBytes;
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk) {
+                            const uint64_t ad = smem_desc_sw128(pa + kk * 32, 16, 1024);
+                            const uint64_t bd = smem_desc_sw128(va + kk * 2048, 8192, 1024);
+                            mma_f16(tmem + 128, ad, bd, IDESC_PV, (npv > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit(pv_done);
+                        mma_commit(v_empty + sp);
+                        ++npv;
+                        progressed = true;
+                    }
+                }
+                if (total >= 0 && npv == total) break;
+                if (!progressed && (++idle & 63) == 0 && (*abort_flag || globaltimer() > deadline)) ok = false;
             }
-            if (ok && n >= 1) ok = issue_pv(n - 1);
             if (!ok) {
                 *abort_flag = 1;
                 record(a.st, SA_ERR_TIMEOUT, CHK_WAIT, 1);
             }
         }
-    } else {
+    } else if (warp >= 2 && warp <= 5) {
         // ------------------------------------------------------------ softmax
         const int q4 = warp & 3;
         const int r = 32 * q4 + lane;
@@ -309,13 +348,10 @@ __global__ void __launch_bounds__(kThreads, 2)
         bool ok = true;
         uint8_t *prow = smem + L::P + r * 128;
         for (;;) {
-            const int s = n % NS;
-            ok = __all_sync(0xffffffffu, mbar_wait(kfull + s, (n / NS) & 1, deadline, abort_flag));
-            if (!ok) break;
-            const int2 sl = make_int2(slots[2 * s], slots[2 * s + 1]);
-            if (sl.x < 0) break;
             ok = __all_sync(0xffffffffu, mbar_wait(s_full + (n & 1), (n >> 1) & 1, deadline, abort_flag));
             if (!ok) break;
+            const int2 sl = make_int2(sinfo[2 * (n & 3)], sinfo[2 * (n & 3) + 1]);
+            if (sl.x < 0) break;
             fence_after_sync();
             const bool sel = (sl.y >> hf) & 1;       // warp-uniform
             uint32_t pk[32];
@@ -329,20 +365,21 @@ __global__ void __launch_bounds__(kThreads, 2)
                 fence_before_sync();
                 mbar_arrive(s_empty + (n & 1));
                 float v[64];
-                float mx = -INFINITY;
                 if (sl.x == iq[hf]) {                // diagonal block: causal inside
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) {
-                        v[c] = c <= rr ? __uint_as_float(sr[c]) : -INFINITY;
-                        mx = fmaxf(mx, v[c]);
-                    }
+                    for (int c = 0; c < 64; ++c) v[c] = c <= rr ? __uint_as_float(sr[c]) : -INFINITY;
                 } else {
 #pragma unroll
-                    for (int c = 0; c < 64; ++c) {
-                        v[c] = __uint_as_float(sr[c]);
-                        mx = fmaxf(mx, v[c]);
-                    }
+                    for (int c = 0; c < 64; ++c) v[c] = __uint_as_float(sr[c]);
                 }
+                // row max with 8 independent chains
+                float m8[8];
+#pragma unroll
+                for (int k = 0; k < 8; ++k) m8[k] = v[k];
+#pragma unroll
+                for (int c = 8; c < 64; ++c) m8[c & 7] = fmaxf(m8[c & 7], v[c]);
+                const float mx = fmaxf(fmaxf(fmaxf(m8[0], m8[1]), fmaxf(m8[2], m8[3])),
+                                       fmaxf(fmaxf(m8[4], m8[5]), fmaxf(m8[6], m8[7])));
                 const float m_new = fmaxf(m_used, mx * C);
                 if (m_new > -INFINITY) {
                     if (m_used == -INFINITY) {
@@ -355,16 +392,19 @@ __global__ void __launch_bounds__(kThreads, 2)
                     }
                 }
                 const float nb = (m_used == -INFINITY) ? 0.f : -m_used;
-                float ps0 = 0.f, ps1 = 0.f;
+                const float2 C2 = make_float2(C, C), nb2 = make_float2(nb, nb);
+                float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                make_float2(0.f, 0.f)};
 #pragma unroll
                 for (int c = 0; c < 64; c += 2) {
-                    const float p0 = ex2(fmaf(v[c], C, nb));
-                    const float p1 = ex2(fmaf(v[c + 1], C, nb));
-                    ps0 += p0;
-                    ps1 += p1;
-                    pk[c >> 1] = pack_bf16x2(p0, p1);
+                    const float2 x = ffma2(make_float2(v[c], v[c + 1]), C2, nb2);
+                    const float2 p = make_float2(ex2(x.x), ex2(x.y));
+                    ps[(c >> 1) & 3] = fadd2(ps[(c >> 1) & 3], p);
+                    pk[c >> 1] = pack_bf16x2(p.x, p.y);
                 }
-                l += ps0 + ps1;
+                const float2 s01 = fadd2(ps[0], ps[1]), s23 = fadd2(ps[2], ps[3]);
+                const float2 s4 = fadd2(s01, s23);
+                l += s4.x + s4.y;
             } else {
                 fence_before_sync();
                 mbar_arrive(s_empty + (n & 1));

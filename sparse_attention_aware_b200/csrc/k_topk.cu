@@ -15,8 +15,9 @@
 // exact radix select on the order-preserving uint32 image of the fp32 score:
 // three digit passes (11, 11, 10 bits) narrow the k-th largest key to a
 // single value T and the number r of elements equal to T that are still to be
-// taken; a final pass emits, in ascending position order, every element
-// above T and the first r elements equal to T (ties to the lower position).
+// taken; the output is every element above T and the first r elements equal
+// to T (ties to the lower position), in ascending position order.  Only the
+// first two passes read the whole row (see the kernel comment).
 #include "sa_internal.h"
 
 namespace sa {
@@ -25,10 +26,35 @@ namespace {
 constexpr int kScoreChunk = 1024;   // tokens per scoring CTA
 constexpr int kSelThreads = 1024;
 
-template <int D, int HPG, bool QF32, int U>
+// Sum N = G values held by each of G lanes across the G lanes so that lane l
+// ends with the full sum of value index (l % G): at every butterfly step a lane
+// keeps the half of its values its lane bit selects and adds the partner's
+// copy of that half (G - 1 shuffles in total instead of N * log2(G)).
+template <int G>
+__device__ __forceinline__ float transpose_reduce(float (&v)[G], int lane)
+{
+#pragma unroll
+    for (int o = G / 2, cnt = G / 2; o >= 1; o >>= 1, cnt >>= 1) {
+        const bool upper = lane & o;
+#pragma unroll
+        for (int i = 0; i < cnt; ++i) {
+            const float send = upper ? v[i] : v[i + cnt];
+            const float keep = upper ? v[i + cnt] : v[i];
+            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+        }
+    }
+    return v[0];
+}
+
+// One group of G = D/8 lanes owns U = G/HPG consecutive token rows per step;
+// the G partial sums (U rows x HPG heads) are reduced with transpose_reduce,
+// after which lane gl holds row gl / HPG, head gl % HPG.
+template <int D, int HPG, bool QF32>
 __global__ void __launch_bounds__(256) k_topk_score(const TopkArgs a)
 {
     constexpr int G = D / 8, GPW = 32 / G, NG = 8 * GPW;
+    constexpr int U = G / HPG;
+    static_assert(U >= 1 && U * HPG == G, "rows per step");
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gl = lane & (G - 1), sub = lane / G;
     const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
@@ -61,6 +87,7 @@ __global__ void __launch_bounds__(256) k_topk_score(const TopkArgs a)
     const int32_t *ptb = a.c.pt + (size_t)b * a.c.max_pages;
     const int Pm = (1 << a.c.Plog2) - 1;
     float *srow = a.scores + ((size_t)b * a.Hq + g * HPG) * a.Lcap;
+    const int my_u = gl / HPG, my_j = gl % HPG;
 
     for (int base0 = t0 + warp * GPW * U; base0 < t1; base0 += NG * U) {
         const int base = base0 + sub * U;
@@ -81,21 +108,26 @@ __global__ void __launch_bounds__(256) k_topk_score(const TopkArgs a)
             const size_t off = ((((size_t)page * a.c.Hkv + g) << a.c.Plog2) + (t & Pm)) * D + gl * 8;
             kr[u] = ok[u] ? ldg_nc_v4(a.c.k + off) : make_uint4(0, 0, 0, 0);
         }
+        float part[G];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            float kf[8] = {bf_lo(kr[u].x), bf_hi(kr[u].x), bf_lo(kr[u].y), bf_hi(kr[u].y),
-                           bf_lo(kr[u].z), bf_hi(kr[u].z), bf_lo(kr[u].w), bf_hi(kr[u].w)};
+            const float kf[8] = {bf_lo(kr[u].x), bf_hi(kr[u].x), bf_lo(kr[u].y), bf_hi(kr[u].y),
+                                 bf_lo(kr[u].z), bf_hi(kr[u].z), bf_lo(kr[u].w), bf_hi(kr[u].w)};
 #pragma unroll
             for (int j = 0; j < HPG; ++j) {
                 float p = qv[j][0] * kf[0];
 #pragma unroll
                 for (int e = 1; e < 8; ++e) p = fmaf(qv[j][e], kf[e], p);
-#pragma unroll
-                for (int o = G / 2; o > 0; o >>= 1) p += __shfl_xor_sync(0xffffffffu, p, o);
-                // an unreadable row (bad page) scores -inf so it is never selected
-                if (gl == j && base + u < t1) srow[(size_t)j * a.Lcap + base + u] = ok[u] ? p : -INFINITY;
+                part[u * HPG + j] = p;
             }
         }
+        const float sc = transpose_reduce<G>(part, gl);
+        const int t = base + my_u;
+        bool okm = false;
+#pragma unroll
+        for (int u = 0; u < U; ++u) okm = (u == my_u) ? ok[u] : okm;
+        // an unreadable row (bad page) scores -inf so it is never selected
+        if (t < t1) srow[(size_t)my_j * a.Lcap + t] = okm ? sc : -INFINITY;
     }
 }
 
@@ -129,15 +161,69 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total)
     return r;
 }
 
+// One radix digit pass over the elements whose key matches (prefix, pmask):
+// histogram of the digit at `shift` (nbits wide), then the digit D holding the
+// need-th largest element; `need` drops by the count above D.
+template <typename KeyAt>
+__device__ void digit_pass(KeyAt key_at, int n, int shift, int nbits, uint32_t &prefix, uint32_t &pmask,
+                           unsigned &need, unsigned *hist, int *warp_tot, unsigned &s_digit, unsigned &s_above)
+{
+    const int tid = threadIdx.x;
+    const int nb = 1 << nbits;
+    for (int i = tid; i < nb; i += kSelThreads) hist[i] = 0;
+    __syncthreads();
+    for (int t = tid; t < n; t += kSelThreads) {
+        const uint32_t key = key_at(t);
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+    }
+    __syncthreads();
+    // thread i owns bins in descending order [nb - (i+1)*per, nb - i*per)
+    const int per = nb / kSelThreads;
+    int mine = 0;
+    for (int j = 0; j < per; ++j) mine += hist[nb - 1 - tid * per - j];
+    int total;
+    const int before = block_excl_scan(mine, warp_tot, total);   // count in higher bins
+    if ((unsigned)before < need && need <= (unsigned)(before + mine)) {
+        int run = before;
+        for (int j = 0; j < per; ++j) {
+            const int bin = nb - 1 - tid * per - j;
+            const int c = hist[bin];
+            if ((unsigned)(run + c) >= need) {
+                s_digit = (unsigned)bin;
+                s_above = (unsigned)run;
+                break;
+            }
+            run += c;
+        }
+    }
+    __syncthreads();
+    need -= s_above;
+    prefix |= s_digit << shift;
+    pmask |= (uint32_t)(nb - 1) << shift;
+    __syncthreads();
+}
+
+constexpr int kCandCap = 4096;
+
+// Exact top-k of one (sequence, query head) score row.  Pass 1 histograms the
+// top 11 bits of the order-preserving key over the whole row; pass 2 reads the
+// row once more, writing a position bitmap of the elements whose top digit is
+// above the threshold digit (warp ballots, no atomics) and collecting the
+// threshold-digit elements as candidates in shared memory.  The remaining 21
+// bits are resolved on the candidates only, and the output is emitted in
+// position order from the bitmaps.  If the candidates overflow their buffer,
+// the remaining digit passes and the emission read the full row instead.
+// Dynamic shared memory: 2 bitmaps of Lcap bits + 2 x kCandCap words.
 __global__ void __launch_bounds__(kSelThreads) k_topk_select(const TopkArgs a)
 {
+    extern __shared__ uint32_t dsm[];
     __shared__ unsigned hist[2048];
     __shared__ int warp_tot[33];
-    __shared__ unsigned s_digit, s_above;
+    __shared__ unsigned s_digit, s_above, s_ncand;
 
     const int row = blockIdx.x;
     const int b = row / a.Hq;
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int Lcap = a.c.max_pages << a.c.Plog2;
     int L = __ldg(a.c.sl + b);
     if (L < 0 || L > Lcap) L = L < 0 ? 0 : Lcap;   // recorded by the scoring kernel
@@ -150,77 +236,120 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const TopkArgs a)
         if (tid == 0) a.cnt[row] = L;
         return;
     }
+    const int nw = (L + 31) >> 5;
+    uint32_t *above = dsm;                 // [nw] elements certainly selected
+    uint32_t *eqmap = dsm + ((Lcap + 31) >> 5);   // [nw] elements equal to the threshold
+    uint32_t *ckey = eqmap + ((Lcap + 31) >> 5);
+    uint32_t *cpos = ckey + kCandCap;
+    auto full_key = [&](int t) { return f2key(__ldcg(sc + t)); };
 
-    // three digit passes over the order-preserving key
     uint32_t prefix = 0, pmask = 0;
     unsigned need = (unsigned)k;
-    const int shifts[3] = {21, 10, 0};
-    const int nbits[3] = {11, 11, 10};
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-        const int shift = shifts[pass];
-        const int nb = 1 << nbits[pass];
-        for (int i = tid; i < nb; i += kSelThreads) hist[i] = 0;
-        __syncthreads();
-        for (int t = tid; t < L; t += kSelThreads) {
-            const uint32_t key = f2key(sc[t]);
-            if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+    digit_pass(full_key, L, 21, 11, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
+    const uint32_t D1 = prefix >> 21;
+
+    // pass 2: bitmap of top digit > D1, candidates with top digit == D1
+    if (tid == 0) s_ncand = 0;
+    __syncthreads();
+    for (int w0 = warp * 32; w0 < nw * 32; w0 += kSelThreads) {
+        const int t = w0 + lane;
+        const uint32_t key = t < L ? full_key(t) : 0u;
+        const uint32_t dg = key >> 21;
+        const unsigned hi = __ballot_sync(0xffffffffu, t < L && dg > D1);
+        const unsigned eq = __ballot_sync(0xffffffffu, t < L && dg == D1);
+        if (lane == 0) {
+            above[w0 >> 5] = hi;
+            eqmap[w0 >> 5] = 0u;
         }
-        __syncthreads();
-        // digit D with count(digit > D) < need <= count(digit >= D):
-        // thread i owns bins in descending order [nb - (i+1)*per, nb - i*per)
-        const int per = nb / kSelThreads;
-        int mine = 0;
-        for (int j = 0; j < per; ++j) mine += hist[nb - 1 - tid * per - j];
-        int total;
-        const int before = block_excl_scan(mine, warp_tot, total);  // count in higher bins
-        if ((unsigned)before < need && need <= (unsigned)(before + mine)) {
-            int run = before;
-            for (int j = 0; j < per; ++j) {
-                const int bin = nb - 1 - tid * per - j;
-                const int c = hist[bin];
-                if ((unsigned)(run + c) >= need) {
-                    s_digit = (unsigned)bin;
-                    s_above = (unsigned)run;
-                    break;
+        if (eq) {
+            unsigned base = 0;
+            if (lane == 0) base = atomicAdd(&s_ncand, (unsigned)__popc(eq));
+            base = __shfl_sync(0xffffffffu, base, 0);
+            if (eq >> lane & 1) {
+                const unsigned slot = base + __popc(eq & ((1u << lane) - 1u));
+                if (slot < kCandCap) {
+                    ckey[slot] = key;
+                    cpos[slot] = (uint32_t)t;
                 }
-                run += c;
             }
         }
-        __syncthreads();
-        need -= s_above;
-        prefix |= s_digit << shift;
-        pmask |= (uint32_t)(nb - 1) << shift;
-        __syncthreads();
     }
-    const uint32_t T = prefix;   // the k-th largest key; take `need` elements equal to T
-
-    // emit in ascending position order
-    int written = 0, eq_seen = 0;
-#pragma unroll 1
-    for (int t0 = 0; t0 < L; t0 += kSelThreads) {
-        const int t = t0 + tid;
-        const uint32_t key = t < L ? f2key(sc[t]) : 0u;
-        const int is_eq = (t < L && key == T) ? 1 : 0;
+    __syncthreads();
+    const unsigned ncand = s_ncand;
+    int written = 0;
+    if (ncand <= kCandCap) {
+        auto cand_key = [&](int i) { return ckey[i]; };
+        digit_pass(cand_key, (int)ncand, 10, 11, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
+        digit_pass(cand_key, (int)ncand, 0, 10, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
+        const uint32_t T = prefix;   // the k-th largest key; take `need` elements equal to T
+        for (int i = tid; i < (int)ncand; i += kSelThreads) {
+            const uint32_t key = ckey[i], t = cpos[i];
+            if (key > T) atomicOr(&above[t >> 5], 1u << (t & 31));
+            else if (key == T) atomicOr(&eqmap[t >> 5], 1u << (t & 31));
+        }
+        __syncthreads();
+        // keep the first `need` equal elements (position order), then emit
+        const int per = (nw + kSelThreads - 1) / kSelThreads;
+        const int w0 = tid * per, w1 = min(w0 + per, nw);
+        int eqc = 0;
+        for (int w = w0; w < w1; ++w) eqc += __popc(eqmap[w]);
         int eq_tot;
-        const int eq_rank = block_excl_scan(is_eq, warp_tot, eq_tot);
-        const int sel = (t < L && (key > T || (is_eq && (unsigned)(eq_seen + eq_rank) < need))) ? 1 : 0;
+        int eq_before = block_excl_scan(eqc, warp_tot, eq_tot);
+        int selc = 0;
+        for (int w = w0; w < w1; ++w) {
+            uint32_t e = eqmap[w];
+            while (e) {
+                const int bit = __ffs(e) - 1;
+                e &= e - 1;
+                if ((unsigned)eq_before < need) above[w] |= 1u << bit;
+                ++eq_before;
+            }
+            selc += __popc(above[w]);
+        }
         int sel_tot;
-        const int pos = block_excl_scan(sel, warp_tot, sel_tot);
-        if (sel) idx[written + pos] = t;
-        written += sel_tot;
-        eq_seen += eq_tot;
+        int pos = block_excl_scan(selc, warp_tot, sel_tot);
+        for (int w = w0; w < w1; ++w) {
+            uint32_t m = above[w];
+            while (m) {
+                const int bit = __ffs(m) - 1;
+                m &= m - 1;
+                if (pos < k) idx[pos] = w * 32 + bit;
+                ++pos;
+            }
+        }
+        written = sel_tot;
+    } else {
+        // candidate overflow (many equal or clustered scores): full-row passes
+        digit_pass(full_key, L, 10, 11, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
+        digit_pass(full_key, L, 0, 10, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
+        const uint32_t T = prefix;
+        int eq_seen = 0;
+#pragma unroll 1
+        for (int t0 = 0; t0 < L; t0 += kSelThreads) {
+            const int t = t0 + tid;
+            const uint32_t key = t < L ? full_key(t) : 0u;
+            const int is_eq = (t < L && key == T) ? 1 : 0;
+            int eq_tot;
+            const int eq_rank = block_excl_scan(is_eq, warp_tot, eq_tot);
+            const int sel = (t < L && (key > T || (is_eq && (unsigned)(eq_seen + eq_rank) < need))) ? 1 : 0;
+            int sel_tot;
+            const int pos = block_excl_scan(sel, warp_tot, sel_tot);
+            if (sel) idx[written + pos] = t;
+            written += sel_tot;
+            eq_seen += eq_tot;
+        }
     }
     if (tid == 0) a.cnt[row] = written;
 }
+
+size_t select_smem_bytes(int Lcap) { return (size_t)2 * ((Lcap + 31) / 32) * 4 + (size_t)2 * kCandCap * 4; }
 
 template <int D, int HPG, bool QF32>
 cudaError_t launch_score(const TopkArgs &a, cudaStream_t s)
 {
     const int Lcap = a.c.max_pages << a.c.Plog2;
     dim3 grid((Lcap + kScoreChunk - 1) / kScoreChunk, a.c.Hkv, a.c.B);
-    constexpr int U = HPG >= 8 ? 2 : 4;
-    k_topk_score<D, HPG, QF32, U><<<grid, 256, 0, s>>>(a);
+    k_topk_score<D, HPG, QF32><<<grid, 256, 0, s>>>(a);
     return cudaGetLastError();
 }
 
@@ -248,7 +377,11 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s)
     else
         e = a.q_f32 ? launch_score_hpg<128, true>(a, hpg, s) : launch_score_hpg<128, false>(a, hpg, s);
     if (e != cudaSuccess) return e;
-    k_topk_select<<<a.c.B * a.Hq, kSelThreads, 0, s>>>(a);
+    const int Lcap = a.c.max_pages << a.c.Plog2;
+    const size_t smem = select_smem_bytes(Lcap);
+    e = cudaFuncSetAttribute(k_topk_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    k_topk_select<<<a.c.B * a.Hq, kSelThreads, smem, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -186,6 +186,8 @@ sa_status sa_select_topk(const sa_kv_cache *kv, const void *q, sa_dtype q_dtype,
     if (hpg != 1 && hpg != 2 && hpg != 4 && hpg != 8) return SA_ERR_UNSUPPORTED;
     if (kv->batch > 0 && (!q || !idx_out || !count_out)) return SA_ERR_INVALID_ARGUMENT;
     if (!aligned(q, 16) || !aligned(idx_out, 4) || !aligned(count_out, 4)) return SA_ERR_INVALID_ARGUMENT;
+    // the selection keeps two bitmaps of the context in shared memory
+    if ((long long)kv->max_pages_per_seq * kv->page_size > (1LL << 19)) return SA_ERR_UNSUPPORTED;
     st = check_ws(ws, ws_bytes, ws_topk(kv, num_q_heads));
     if (st != SA_OK) return st;
     a.q = q;
