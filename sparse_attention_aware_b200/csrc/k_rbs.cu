@@ -13,24 +13,28 @@
 //                  shared memory).
 //   k_pool_q       per (query block i, q head h): qbar_i = mean of the block's
 //                  queries, ||qbar_i||.
-//   k_pair_tile    per (64x64 tile of causal block pairs, q head): the pooled
+//   k_pair_tile    per (128x128 tile of causal block pairs, q head): the pooled
 //                  dot products qbar_i . c_j (fp32 SIMT tile product), both
 //                  branch scores, thresholds, OR with the forced diagonal and
 //                  first block -> mask bits and per-row counts.  In quantile
 //                  mode the scores are stored instead and
-//   k_quantile     finds each head's lower quantile (exact radix select on the
-//                  order-preserving key) and
+//   k_qhist/k_qpick  find each head's lower quantile (exact radix select on
+//                  the order-preserving key, grid-wide histograms) and
 //   k_mask_scores  thresholds the stored scores.
 //   k_csr_scan / k_csr_fill  turn counts and bits into CSR (ascending cols).
 #include "sa_internal.h"
 
 namespace sa {
 
+namespace {
+// mask bit words per (head, query block) row: 4 per 128-wide tile column
+__host__ __device__ inline int mask_words(int nB) { return 4 * ((nB + 127) / 128); }
+}  // namespace
+
 size_t rbs_workspace_layout(int Hq, int Hkv, int D, int nB, bool quantile, size_t *offs)
 {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-    const size_t nTB = (nB + 63) / 64;
-    const size_t words = 2 * nTB;
+    const size_t words = mask_words(nB);
     const size_t nP = (size_t)nB * (nB + 1) / 2;
     size_t o = 0;
     offs[0] = o; o += up((size_t)Hkv * nB * D * 4);       // centroids
@@ -39,9 +43,11 @@ size_t rbs_workspace_layout(int Hq, int Hkv, int D, int nB, bool quantile, size_
     offs[3] = o; o += up((size_t)Hq * nB * 4);            // pooled query norms
     offs[4] = o; o += up((size_t)2 * Hq * 4);             // thresholds
     offs[5] = o; o += up((size_t)Hq * nB * words * 4);    // mask bits
-    offs[6] = o; o += up((size_t)Hq * nB * 4 + 4);        // row counts
+    offs[6] = o; o += up((size_t)Hq * nB * 4 + 16 + ((size_t)Hq * nB / 1024 + 2) * 8);   // row counts + chunk sums
     offs[7] = o; if (quantile) o += up((size_t)2 * Hq * nP * 4);   // pair scores
-    offs[8] = o; if (quantile) o += up((size_t)2 * Hq * 4);        // unused scratch
+    // radix-select scratch: per (branch, head) a 2048-bin histogram for each of
+    // the 3 digit passes + state {prefix, mask, need}
+    offs[8] = o; if (quantile) o += up((size_t)2 * Hq * (3 * 2048 + 4) * 4);
     return o;
 }
 
@@ -149,79 +155,97 @@ __device__ __forceinline__ void tri_index(int x, int &I, int &J)
     J = x - r * (r + 1) / 2;
 }
 
+// 128 x 128 tile of causal block pairs of one head: qbar_i . c_j for i in the
+// row tile I, j in the column tile J <= I (fp32 SIMT: 256 threads, 8 x 8
+// outputs each, K staged through shared memory in chunks of 32, transposed so
+// each thread reads its 8 rows and 8 columns with two 16-byte loads each).
+constexpr int kPT = 128;   // tile edge (blocks)
+constexpr int kPK = 32;    // K chunk
+
 template <bool QUANT>
 __global__ void __launch_bounds__(256) k_pair_tile(const RbsArgs a)
 {
     constexpr int D = 128;
-    extern __shared__ __align__(16) float smem[];
-    float *sQ = smem;             // [D][64] transposed pooled queries
-    float *sC = smem + D * 64;    // [D][64] transposed centroids
+    __shared__ __align__(16) float sQ[kPK][kPT];
+    __shared__ __align__(16) float sC[kPK][kPT];
     int I, J;
     tri_index(blockIdx.x, I, J);
     const int h = blockIdx.y;
     const int g = h / (a.Hq / a.c.Hkv);
     const int tid = threadIdx.x;
-    // load the two 64 x 128 fp32 tiles, transposed
-    for (int x = tid; x < 64 * (D / 4); x += 256) {
-        const int r = x & 63, kq = x >> 6;     // row, float4 column index
-        const int i = I * 64 + r, j = J * 64 + r;
-        float4 qv = make_float4(0, 0, 0, 0), cv = make_float4(0, 0, 0, 0);
-        if (i < a.nB) qv = *reinterpret_cast<const float4 *>(a.qbar + ((size_t)h * a.nB + i) * D + kq * 4);
-        if (j < a.nB) cv = *reinterpret_cast<const float4 *>(a.cen + ((size_t)g * a.nB + j) * D + kq * 4);
-        sQ[(kq * 4 + 0) * 64 + r] = qv.x; sQ[(kq * 4 + 1) * 64 + r] = qv.y;
-        sQ[(kq * 4 + 2) * 64 + r] = qv.z; sQ[(kq * 4 + 3) * 64 + r] = qv.w;
-        sC[(kq * 4 + 0) * 64 + r] = cv.x; sC[(kq * 4 + 1) * 64 + r] = cv.y;
-        sC[(kq * 4 + 2) * 64 + r] = cv.z; sC[(kq * 4 + 3) * 64 + r] = cv.w;
-    }
-    __syncthreads();
     const int ty = tid >> 4, tx = tid & 15;
-    float acc[4][4];
+    float acc[8][8];
 #pragma unroll
-    for (int r = 0; r < 4; ++r)
+    for (int r = 0; r < 8; ++r)
 #pragma unroll
-        for (int c = 0; c < 4; ++c) acc[r][c] = 0.f;
-#pragma unroll 8
-    for (int k = 0; k < D; ++k) {
-        const float4 qa = *reinterpret_cast<const float4 *>(&sQ[k * 64 + ty * 4]);
-        const float4 cb = *reinterpret_cast<const float4 *>(&sC[k * 64 + tx * 4]);
-        const float qr[4] = {qa.x, qa.y, qa.z, qa.w};
-        const float cr[4] = {cb.x, cb.y, cb.z, cb.w};
+        for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
+    const float *qb = a.qbar + (size_t)h * a.nB * D;
+    const float *cb = a.cen + (size_t)g * a.nB * D;
+#pragma unroll 1
+    for (int k0 = 0; k0 < D; k0 += kPK) {
+        for (int x = tid; x < kPT * (kPK / 4); x += 256) {
+            const int r = x & (kPT - 1), kq = x >> 7;   // row in tile, float4 index in chunk
+            const int i = I * kPT + r, j = J * kPT + r;
+            float4 qv = make_float4(0, 0, 0, 0), cv = make_float4(0, 0, 0, 0);
+            if (i < a.nB) qv = *reinterpret_cast<const float4 *>(qb + (size_t)i * D + k0 + kq * 4);
+            if (j < a.nB) cv = *reinterpret_cast<const float4 *>(cb + (size_t)j * D + k0 + kq * 4);
+            sQ[kq * 4 + 0][r] = qv.x; sQ[kq * 4 + 1][r] = qv.y; sQ[kq * 4 + 2][r] = qv.z; sQ[kq * 4 + 3][r] = qv.w;
+            sC[kq * 4 + 0][r] = cv.x; sC[kq * 4 + 1][r] = cv.y; sC[kq * 4 + 2][r] = cv.z; sC[kq * 4 + 3][r] = cv.w;
+        }
+        __syncthreads();
+#pragma unroll 4
+        for (int k = 0; k < kPK; ++k) {
+            const float4 q0 = *reinterpret_cast<const float4 *>(&sQ[k][ty * 8]);
+            const float4 q1 = *reinterpret_cast<const float4 *>(&sQ[k][ty * 8 + 4]);
+            const float4 c0 = *reinterpret_cast<const float4 *>(&sC[k][tx * 8]);
+            const float4 c1 = *reinterpret_cast<const float4 *>(&sC[k][tx * 8 + 4]);
+            const float qr[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
+            const float cr[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
 #pragma unroll
-        for (int r = 0; r < 4; ++r)
+            for (int r = 0; r < 8; ++r)
 #pragma unroll
-            for (int c = 0; c < 4; ++c) acc[r][c] = fmaf(qr[r], cr[c], acc[r][c]);
+                for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(qr[r], cr[c], acc[r][c]);
+        }
+        __syncthreads();
     }
     const float tc = QUANT ? 0.f : __ldg(a.tau_c + h);
     const float tr = QUANT ? 0.f : __ldg(a.tau_r + h);
     const size_t nP = (size_t)a.nB * (a.nB + 1) / 2;
+    const int words = mask_words(a.nB);
+    float rj[8];
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int i = I * 64 + ty * 4 + r;
+    for (int c = 0; c < 8; ++c) {
+        const int j = J * kPT + tx * 8 + c;
+        rj[c] = j < a.nB ? a.rad[(size_t)g * a.nB + j] : 0.f;
+    }
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+        const int i = I * kPT + ty * 8 + r;
         const float qn = i < a.nB ? a.qnorm[(size_t)h * a.nB + i] : 0.f;
-        uint32_t nib = 0;
+        uint32_t byte = 0;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-            const int j = J * 64 + tx * 4 + c;
+        for (int c = 0; c < 8; ++c) {
+            const int j = J * kPT + tx * 8 + c;
             if (i >= a.nB || j > i) continue;
             const float qc = acc[r][c];
             const float sc = a.scale * qc;
-            const float sr = a.scale * fmaf(qn, a.rad[(size_t)g * a.nB + j], qc);
+            const float sr = a.scale * fmaf(qn, rj[c], qc);
             if (QUANT) {
                 const size_t p = (size_t)i * (i + 1) / 2 + j;
                 a.pair_sc[(size_t)h * nP + p] = sc;
                 a.pair_sc[((size_t)a.Hq + h) * nP + p] = sr;
             } else {
                 const bool keep = sc > tc || sr > tr || (a.force_diag && j == i) || (a.force_first && j == 0);
-                nib |= (uint32_t)keep << c;
+                byte |= (uint32_t)keep << c;
             }
         }
         if (!QUANT) {
-            uint32_t w = nib << ((tx & 7) * 4);
-#pragma unroll
-            for (int o = 1; o < 8; o <<= 1) w |= __shfl_xor_sync(0xffffffffu, w, o);
-            if ((tx & 7) == 0 && i < a.nB) {
-                const int words = 2 * ((a.nB + 63) / 64);
-                a.bits[((size_t)h * a.nB + i) * words + J * 2 + (tx >> 3)] = w;
+            // word = 4 consecutive tx (32 columns); lanes tx..tx+3 are adjacent
+            uint32_t w = byte << ((tx & 3) * 8);
+            w |= __shfl_xor_sync(0xffffffffu, w, 1);
+            w |= __shfl_xor_sync(0xffffffffu, w, 2);
+            if ((tx & 3) == 0 && i < a.nB) {
+                a.bits[((size_t)h * a.nB + i) * words + J * 4 + (tx >> 2)] = w;
                 if (w) atomicAdd(&a.rowcnt[h * a.nB + i], __popc(w));
             }
         }
@@ -259,61 +283,109 @@ __device__ __forceinline__ long long block_excl_scan_ll(long long v, long long *
     return r;
 }
 
-// Lower quantile: the element at ascending rank floor(p*(n-1)) among head h's
-// causal pair scores of one branch (exact, three radix digit passes).
-__global__ void __launch_bounds__(1024) k_quantile(const RbsArgs a)
+// Lower quantile of each (branch, head)'s causal pair scores, the element at
+// ascending rank floor(p*(n-1)): an exact radix select on the order-preserving
+// key in three digit passes (11, 11, 10 bits).  Each pass is a grid-wide
+// histogram (k_qhist: many CTAs per score array, shared-memory histograms
+// flushed to global memory) followed by a one-CTA digit pick (k_qpick) that
+// narrows (prefix, mask, need).  Scratch per array: 3 x 2048 bins + state.
+constexpr int kQChunk = 1 << 17;   // scores per histogram CTA
+
+__device__ __forceinline__ uint32_t *qhist_of(const RbsArgs &a, int arr, int pass)
+{
+    return a.qhist + (size_t)arr * (3 * 2048 + 4) + pass * 2048;
+}
+__device__ __forceinline__ uint32_t *qstate_of(const RbsArgs &a, int arr)
+{
+    return a.qhist + (size_t)arr * (3 * 2048 + 4) + 3 * 2048;
+}
+
+__global__ void __launch_bounds__(512) k_qhist(const RbsArgs a, int pass)
 {
     __shared__ unsigned hist[2048];
+    const int arr = blockIdx.y;          // branch * Hq + h
+    const size_t nP = (size_t)a.nB * (a.nB + 1) / 2;
+    const size_t t0 = (size_t)blockIdx.x * kQChunk;
+    if (t0 >= nP) return;
+    const size_t t1 = min(t0 + (size_t)kQChunk, nP);
+    const int shift = pass == 0 ? 21 : pass == 1 ? 10 : 0;
+    const int nb = pass == 2 ? 1024 : 2048;
+    uint32_t prefix = 0, pmask = 0;
+    if (pass > 0) {
+        const uint32_t *st = qstate_of(a, arr);
+        prefix = st[0];
+        pmask = st[1];
+    }
+    for (int i = threadIdx.x; i < nb; i += blockDim.x) hist[i] = 0;
+    __syncthreads();
+    const float *x = a.pair_sc + (size_t)arr * nP;
+    for (size_t t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
+        const uint32_t key = f2key(__ldcs(x + t));
+        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+    }
+    __syncthreads();
+    uint32_t *gh = qhist_of(a, arr, pass);
+    for (int i = threadIdx.x; i < nb; i += blockDim.x)
+        if (hist[i]) atomicAdd(&gh[i], hist[i]);
+}
+
+__global__ void __launch_bounds__(1024) k_qpick(const RbsArgs a, int pass)
+{
     __shared__ long long wt[33];
     __shared__ unsigned s_digit;
     __shared__ long long s_below;
-    const int branch = blockIdx.x / a.Hq, h = blockIdx.x % a.Hq;
+    const int arr = blockIdx.x;
+    const int branch = arr / a.Hq, h = arr % a.Hq;
     const size_t nP = (size_t)a.nB * (a.nB + 1) / 2;
-    const float *x = a.pair_sc + ((size_t)branch * a.Hq + h) * nP;
-    const float p = branch == 0 ? a.p_c : a.p_r;
-    long long need = (long long)floor((double)p * (double)(nP - 1)) + 1;   // 1-based ascending rank
+    uint32_t *st = qstate_of(a, arr);
     uint32_t prefix = 0, pmask = 0;
-    const int shifts[3] = {21, 10, 0}, nbits[3] = {11, 11, 10};
-#pragma unroll 1
-    for (int pass = 0; pass < 3; ++pass) {
-        const int shift = shifts[pass], nb = 1 << nbits[pass];
-        for (int t = threadIdx.x; t < nb; t += blockDim.x) hist[t] = 0;
-        __syncthreads();
-        for (size_t t = threadIdx.x; t < nP; t += blockDim.x) {
-            const uint32_t key = f2key(x[t]);
-            if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
-        }
-        __syncthreads();
-        const int per = nb / blockDim.x;
-        long long mine = 0;
-        for (int q = 0; q < per; ++q) mine += hist[threadIdx.x * per + q];
-        long long total;
-        const long long before = block_excl_scan_ll(mine, wt, total);   // count in lower digits
-        if (before < need && need <= before + mine) {
-            long long run = before;
-            for (int q = 0; q < per; ++q) {
-                const int bin = threadIdx.x * per + q;
-                if (run + hist[bin] >= need) {
-                    s_digit = (unsigned)bin;
-                    s_below = run;
-                    break;
-                }
-                run += hist[bin];
+    long long need;
+    if (pass == 0) {
+        const float p = branch == 0 ? a.p_c : a.p_r;
+        need = (long long)floor((double)p * (double)(nP - 1)) + 1;   // 1-based ascending rank
+    } else {
+        prefix = st[0];
+        pmask = st[1];
+        need = (long long)st[2] | ((long long)st[3] << 32);
+    }
+    const int shift = pass == 0 ? 21 : pass == 1 ? 10 : 0;
+    const int nb = pass == 2 ? 1024 : 2048;
+    const uint32_t *hist = qhist_of(a, arr, pass);
+    const int per = nb / blockDim.x;
+    long long mine = 0;
+    for (int q = 0; q < per; ++q) mine += hist[threadIdx.x * per + q];
+    long long total;
+    const long long before = block_excl_scan_ll(mine, wt, total);   // count in lower digits
+    if (before < need && need <= before + mine) {
+        long long run = before;
+        for (int q = 0; q < per; ++q) {
+            const int bin = threadIdx.x * per + q;
+            if (run + hist[bin] >= need) {
+                s_digit = (unsigned)bin;
+                s_below = run;
+                break;
             }
+            run += hist[bin];
         }
-        __syncthreads();
+    }
+    __syncthreads();
+    if (threadIdx.x == 0) {
         need -= s_below;
         prefix |= s_digit << shift;
         pmask |= (uint32_t)(nb - 1) << shift;
-        __syncthreads();
-    }
-    if (threadIdx.x == 0) {
-        const uint32_t u = (prefix & 0x80000000u) ? (prefix & 0x7fffffffu) : ~prefix;
-        a.tau[branch * a.Hq + h] = __uint_as_float(u);
+        st[0] = prefix;
+        st[1] = pmask;
+        st[2] = (uint32_t)(need & 0xffffffffu);
+        st[3] = (uint32_t)(need >> 32);
+        if (pass == 2) {
+            const uint32_t u = (prefix & 0x80000000u) ? (prefix & 0x7fffffffu) : ~prefix;
+            a.tau[branch * a.Hq + h] = __uint_as_float(u);
+        }
     }
 }
 
-// quantile mode: threshold the stored pair scores; one warp per row (h, i)
+// quantile mode: threshold the stored pair scores; one warp per row (h, i),
+// four 32-column words in flight per iteration
 __global__ void __launch_bounds__(256) k_mask_scores(const RbsArgs a)
 {
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
@@ -324,37 +396,71 @@ __global__ void __launch_bounds__(256) k_mask_scores(const RbsArgs a)
     const float *sc = a.pair_sc + (size_t)h * nP + (size_t)i * (i + 1) / 2;
     const float *sr = a.pair_sc + ((size_t)a.Hq + h) * nP + (size_t)i * (i + 1) / 2;
     const float tc = a.tau[h], tr = a.tau[a.Hq + h];
-    const int words = 2 * ((a.nB + 63) / 64);
+    const int words = mask_words(a.nB);
+    const int nw = i / 32 + 1;
     int cnt = 0;
-    for (int w0 = 0; w0 <= i / 32; ++w0) {
-        const int j = w0 * 32 + lane;
-        bool keep = false;
-        if (j <= i) keep = sc[j] > tc || sr[j] > tr || (a.force_diag && j == i) || (a.force_first && j == 0);
-        const uint32_t w = __ballot_sync(0xffffffffu, keep);
-        if (lane == 0) a.bits[(size_t)row * words + w0] = w;
-        cnt += __popc(w);
+    for (int w0 = 0; w0 < nw; w0 += 4) {
+        float vc[4], vr[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = (w0 + u) * 32 + lane;
+            vc[u] = j <= i ? __ldcs(sc + j) : 0.f;
+            vr[u] = j <= i ? __ldcs(sr + j) : 0.f;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int j = (w0 + u) * 32 + lane;
+            const bool keep = j <= i && (vc[u] > tc || vr[u] > tr || (a.force_diag && j == i) ||
+                                         (a.force_first && j == 0));
+            const uint32_t w = __ballot_sync(0xffffffffu, keep);
+            if (lane == 0 && w0 + u < nw) a.bits[(size_t)row * words + w0 + u] = w;
+            cnt += __popc(w);
+        }
     }
     if (lane == 0) a.rowcnt[row] = cnt;
 }
 
-__global__ void __launch_bounds__(1024) k_csr_scan(const RbsArgs a)
+// CSR row pointers: exclusive prefix sum of the row counts in three short
+// launches (per-chunk sums, one scan of the chunk sums, per-chunk write-out).
+constexpr int kScanChunk = 1024;   // rows per CTA (one per thread)
+
+__global__ void __launch_bounds__(kScanChunk) k_csr_sum(const RbsArgs a, long long *chunk_sum)
 {
     __shared__ long long wt[33];
     const int R = a.Hq * a.nB;
-    const int per = (R + blockDim.x - 1) / blockDim.x;
-    const int r0 = threadIdx.x * per, r1 = min(r0 + per, R);
-    long long s = 0;
-    for (int r = r0; r < r1; ++r) s += a.rowcnt[r];
+    const int r = blockIdx.x * kScanChunk + threadIdx.x;
     long long total;
-    long long run = block_excl_scan_ll(s, wt, total);
-    for (int r = r0; r < r1; ++r) {
-        a.row_ptr[r] = (int32_t)min(run, (long long)INT32_MAX);
-        run += a.rowcnt[r];
+    block_excl_scan_ll(r < R ? a.rowcnt[r] : 0, wt, total);
+    if (threadIdx.x == 0) chunk_sum[blockIdx.x] = total;
+}
+
+__global__ void __launch_bounds__(1024) k_csr_chunks(const RbsArgs a, long long *chunk_sum, int nchunks)
+{
+    __shared__ long long wt[33];
+    long long run = 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 1024) {
+        const int c = c0 + threadIdx.x;
+        const long long v = c < nchunks ? chunk_sum[c] : 0;
+        long long total;
+        const long long ex = block_excl_scan_ll(v, wt, total);
+        if (c < nchunks) chunk_sum[c] = run + ex;
+        run += total;
     }
     if (threadIdx.x == 0) {
-        a.row_ptr[R] = (int32_t)min(total, (long long)INT32_MAX);
-        if (total > a.nnz_cap) record(a.st, SA_ERR_CAPACITY, CHK_CAPACITY_CSR, (int)min(total, (long long)INT32_MAX));
+        const int R = a.Hq * a.nB;
+        a.row_ptr[R] = (int32_t)min(run, (long long)INT32_MAX);
+        if (run > a.nnz_cap) record(a.st, SA_ERR_CAPACITY, CHK_CAPACITY_CSR, (int)min(run, (long long)INT32_MAX));
     }
+}
+
+__global__ void __launch_bounds__(kScanChunk) k_csr_scan(const RbsArgs a, const long long *chunk_off)
+{
+    __shared__ long long wt[33];
+    const int R = a.Hq * a.nB;
+    const int r = blockIdx.x * kScanChunk + threadIdx.x;
+    long long total;
+    const long long ex = block_excl_scan_ll(r < R ? a.rowcnt[r] : 0, wt, total);
+    if (r < R) a.row_ptr[r] = (int32_t)min(chunk_off[blockIdx.x] + ex, (long long)INT32_MAX);
 }
 
 __global__ void __launch_bounds__(256) k_csr_fill(const RbsArgs a)
@@ -363,7 +469,7 @@ __global__ void __launch_bounds__(256) k_csr_fill(const RbsArgs a)
     const int lane = threadIdx.x & 31;
     if (row >= a.Hq * a.nB) return;
     const int i = row % a.nB;
-    const int words = 2 * ((a.nB + 63) / 64);
+    const int words = mask_words(a.nB);
     const int nw = i / 32 + 1;
     long long base = a.row_ptr[row];
     for (int w0 = 0; w0 < nw; w0 += 32) {
@@ -414,22 +520,33 @@ cudaError_t launch_rbs(const RbsArgs &a, cudaStream_t s)
     k_block_stats<<<dim3(a.nB, a.c.Hkv), 256, 0, s>>>(a);
     k_pool_q<<<dim3(a.nB, a.Hq), 256, 0, s>>>(a);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const int nTB = (a.nB + 63) / 64;
+    const int nTB = (a.nB + kPT - 1) / kPT;
     const int tiles = nTB * (nTB + 1) / 2;
-    const size_t smem = 2 * 128 * 64 * sizeof(float);
+    const size_t smem = 0;
     if (quant) {
-        cudaFuncSetAttribute(k_pair_tile<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k_pair_tile<true><<<dim3(tiles, a.Hq), 256, smem, s>>>(a);
-        k_quantile<<<2 * a.Hq, 1024, 0, s>>>(a);
+        if ((e = cudaMemsetAsync(a.qhist, 0, (size_t)2 * a.Hq * (3 * 2048 + 4) * 4, s)) != cudaSuccess) return e;
+        const size_t nP = (size_t)a.nB * (a.nB + 1) / 2;
+        const dim3 hgrid((unsigned)((nP + kQChunk - 1) / kQChunk), 2 * a.Hq);
+        for (int pass = 0; pass < 3; ++pass) {
+            k_qhist<<<hgrid, 512, 0, s>>>(a, pass);
+            k_qpick<<<2 * a.Hq, 1024, 0, s>>>(a, pass);
+        }
         k_mask_scores<<<(a.Hq * a.nB + 7) / 8, 256, 0, s>>>(a);
     } else {
-        cudaFuncSetAttribute(k_pair_tile<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
         k_copy_tau<<<(a.Hq + 127) / 128, 128, 0, s>>>(a);
         if ((e = cudaMemsetAsync(a.rowcnt, 0, (size_t)a.Hq * a.nB * sizeof(int32_t), s)) != cudaSuccess) return e;
         k_pair_tile<false><<<dim3(tiles, a.Hq), 256, smem, s>>>(a);
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    k_csr_scan<<<1, 1024, 0, s>>>(a);
+    {
+        const int R = a.Hq * a.nB;
+        const int nch = (R + kScanChunk - 1) / kScanChunk;
+        long long *chunk = reinterpret_cast<long long *>(a.rowcnt + R + 1 + ((R + 1) & 1));   // 8-byte aligned
+        k_csr_sum<<<nch, kScanChunk, 0, s>>>(a, chunk);
+        k_csr_chunks<<<1, 1024, 0, s>>>(a, chunk, nch);
+        k_csr_scan<<<nch, kScanChunk, 0, s>>>(a, chunk);
+    }
     k_csr_fill<<<(a.Hq * a.nB + 7) / 8, 256, 0, s>>>(a);
     if (a.tau_out) k_tau_out<<<(2 * a.Hq + 127) / 128, 128, 0, s>>>(a);
     return cudaGetLastError();

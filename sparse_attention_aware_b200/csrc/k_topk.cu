@@ -23,7 +23,7 @@
 namespace sa {
 namespace {
 
-constexpr int kScoreChunk = 1024;   // tokens per scoring CTA
+constexpr int kScoreChunk = 4096;   // tokens per scoring CTA
 constexpr int kSelThreads = 1024;
 
 // Sum N = G values held by each of G lanes across the G lanes so that lane l
