@@ -15,26 +15,25 @@
 //   warp 0      K producer: the Q halves (3-D map over [T][Hq][128]), then
 //               per key block of the merged list the K page tile (2-D map over
 //               the paged cache; page table resolved per block), 128-byte
-//               swizzle, NS-stage ring released as soon as S = QK^T of that
+//               swizzle, 3-stage ring released as soon as S = QK^T of that
 //               block has completed.  It merges the two CSR rows and posts
 //               (block, half mask) per stage, with an end sentinel.
 //   warp 6      V producer: the V page tiles of the same merged list into their
-//               own NS-stage ring, released when PV of that block completes.
+//               own 2-stage ring, released when PV of that block completes.
 //   warp 1      MMA issuer (one thread) and TMEM owner: S = Q K^T (M=128, N=64,
-//               K=128) into one of two TMEM S buffers, O += P V (M=128, N=128,
-//               K=64) into the TMEM O accumulator.  S runs up to two blocks
-//               ahead of PV (S_0 S_1 S_2 PV_0 S_3 PV_1 ...); the thread polls
-//               the readiness of the next S and the next PV so neither blocks
-//               the other.  It forwards each block's (index, half mask) to the
-//               softmax through a shared ring published by a release-arrive on
-//               the S-ready barrier.
+//               K=128) into one of two TMEM S buffers; O += P V (M=128, N=128,
+//               K=64) with P read from TMEM, where the softmax wrote it over
+//               the first 32 columns of S's buffer; order S_0, S_1, PV_0, S_2,
+//               PV_1, S_3, ...  It forwards each block's (index, half mask) to
+//               the softmax through a shared ring published by a release-arrive
+//               on the S-ready barrier.
 //   warps 2-5   softmax: one query row per thread (TMEM lane); half-selection
 //               and causal masks (only the diagonal block needs per-element
 //               masking); base-2 online softmax with the scale folded into the
 //               exponent's FMA and lazy rescaling (O and l rescaled only when
-//               the running max grows by more than 2^8); P written to shared
-//               memory as bf16 in the swizzled K-major layout the PV MMA reads;
-//               final O / l -> bf16 and LSE.
+//               the running max grows by more than 2^8); P written to TMEM as
+//               bf16 pairs; it waits for PV only before a rescale of O and at
+//               the end; final O / l -> bf16 and LSE.
 // Every wait is bounded (globaltimer deadline, shared abort flag): on expiry
 // the kernel records SA_ERR_TIMEOUT, drains its own outstanding copies and
 // MMAs with bounded waits, frees its TMEM and returns.
@@ -61,26 +60,24 @@ namespace {
 using namespace tc;
 
 constexpr int kThreads = 224;
-constexpr int kTmemCols = 256;                 // S0 [0,64) S1 [64,128) O [128,256)
+constexpr int kTmemCols = 256;                 // S0/P0 [0,64) S1/P1 [64,128) O [128,256)
 constexpr uint32_t kQBytes = 128 * 128 * 2;     // 32 KB
 constexpr uint32_t kKVBytes = 64 * 128 * 2;     // 16 KB per K (or V) block
-constexpr uint32_t kPBytes = 128 * 64 * 2;      // 16 KB
 constexpr uint64_t kWaitNs = 400ull * 1000 * 1000;   // 0.4 s
 
 constexpr uint32_t IDESC_S = idesc_bf16(128, 64, 0, 0);
 constexpr uint32_t IDESC_PV = idesc_bf16(128, 128, 0, 1);
 
-template <int NS>
+template <int NSK, int NSV>
 struct Smem {
     static constexpr uint32_t Q = 0;
     static constexpr uint32_t K = Q + kQBytes;
-    static constexpr uint32_t V = K + NS * kKVBytes;
-    static constexpr uint32_t P = V + NS * kKVBytes;
-    static constexpr uint32_t BAR = P + kPBytes;
-    // q_full, kfull[NS], vfull[NS], k_empty[NS], v_empty[NS], s_full[2], s_empty[2], p_full, pv_done
-    static constexpr int NBAR = 1 + 4 * NS + 6;
-    static constexpr uint32_t SLOT = BAR + NBAR * 8;       // int2 slot[NS]: K producer -> MMA
-    static constexpr uint32_t SINFO = SLOT + NS * 8;       // int2 sinfo[4]: MMA -> softmax
+    static constexpr uint32_t V = K + NSK * kKVBytes;
+    static constexpr uint32_t BAR = V + NSV * kKVBytes;
+    // q_full, kfull[NSK], k_empty[NSK], vfull[NSV], v_empty[NSV], s_full[2], p_full[2], pv_done
+    static constexpr int NBAR = 1 + 2 * NSK + 2 * NSV + 5;
+    static constexpr uint32_t SLOT = BAR + NBAR * 8;       // int2 slot[NSK]: K producer -> MMA
+    static constexpr uint32_t SINFO = SLOT + NSK * 8;      // int2 sinfo[4]: MMA -> softmax
     static constexpr uint32_t MISC = SINFO + 4 * 8;
     static constexpr uint32_t TOTAL = MISC + 16;
 };
@@ -134,12 +131,12 @@ struct Merge {
     }
 };
 
-template <int NS>
+template <int NSK, int NSV>
 __global__ void __launch_bounds__(kThreads, 2)
     k_prefill_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const PrefillArgs a)
 {
-    using L = Smem<NS>;
+    using L = Smem<NSK, NSV>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
     if (sbase & 1023u) {   // uniform for the whole CTA
@@ -149,13 +146,12 @@ __global__ void __launch_bounds__(kThreads, 2)
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + L::BAR);
     uint64_t *q_full = bars;
     uint64_t *kfull = bars + 1;
-    uint64_t *vfull = kfull + NS;
-    uint64_t *k_empty = vfull + NS;
-    uint64_t *v_empty = k_empty + NS;
-    uint64_t *s_full = v_empty + NS;
-    uint64_t *s_empty = s_full + 2;
-    uint64_t *p_full = s_empty + 2;
-    uint64_t *pv_done = p_full + 1;
+    uint64_t *k_empty = kfull + NSK;
+    uint64_t *vfull = k_empty + NSK;
+    uint64_t *v_empty = vfull + NSV;
+    uint64_t *s_full = v_empty + NSV;
+    uint64_t *p_full = s_full + 2;     // per S buffer: the softmax may run one block ahead
+    uint64_t *pv_done = p_full + 2;
     volatile int *slots = reinterpret_cast<volatile int *>(smem + L::SLOT);   // (j, mask) per K stage
     volatile int *sinfo = reinterpret_cast<volatile int *>(smem + L::SINFO); // (j, mask) per S, ring of 4
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + L::MISC);
@@ -171,17 +167,18 @@ __global__ void __launch_bounds__(kThreads, 2)
 
     if (threadIdx.x == 0) {
         mbar_init(q_full, 1);
-        for (int s = 0; s < NS; ++s) {
+        for (int s = 0; s < NSK; ++s) {
             mbar_init(kfull + s, 1);
-            mbar_init(vfull + s, 1);
             mbar_init(k_empty + s, 1);
+        }
+        for (int s = 0; s < NSV; ++s) {
+            mbar_init(vfull + s, 1);
             mbar_init(v_empty + s, 1);
         }
         for (int b = 0; b < 2; ++b) {
-            mbar_init(s_full + b, 2);      // S MMAs complete + block info posted
-            mbar_init(s_empty + b, 128);
+            mbar_init(s_full + b, 2);
+            mbar_init(p_full + b, 128);
         }
-        mbar_init(p_full, 128);
         mbar_init(pv_done, 1);
         *abort_flag = 0;
         fence_mbar_init();
@@ -216,6 +213,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         // ------------------------------------------------------ K / V producers
         if (lane == 0) {
             const bool is_k = warp == 0;
+            const int NS = is_k ? NSK : NSV;
             uint64_t *full = is_k ? kfull : vfull;
             uint64_t *empty = is_k ? k_empty : v_empty;
             const CUtensorMap *map = is_k ? &tmK : &tmV;
@@ -269,65 +267,56 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------ MMA
+        // order: S_0, S_1, then PV_n, S_{n+2}, PV_{n+1}, S_{n+3}, ...  P_n lives
+        // in TMEM over S_n's columns, so S_{n+2} (same buffer) follows PV_n.
         if (lane == 0) {
             const uint32_t qa = sbase + L::Q;
-            const uint32_t pa = sbase + L::P;
+            int ns = 0, total = -1;
+            auto issue_s = [&]() -> bool {
+                const int s = ns % NSK;
+                if (!mbar_wait(kfull + s, (ns / NSK) & 1, deadline, abort_flag)) return false;
+                const int j = slots[2 * s], m = slots[2 * s + 1];
+                sinfo[2 * (ns & 3)] = j;
+                sinfo[2 * (ns & 3) + 1] = m;
+                if (j < 0) {
+                    total = ns;
+                    mbar_arrive(s_full + (ns & 1));
+                    mbar_arrive(s_full + (ns & 1));
+                    return true;
+                }
+                fence_after_sync();
+                const uint32_t ka = sbase + L::K + s * kKVBytes;
+#pragma unroll
+                for (int kk = 0; kk < 8; ++kk) {
+                    const uint64_t ad = smem_desc_sw128(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
+                    const uint64_t bd = smem_desc_sw128(ka + (kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32, 16, 1024);
+                    mma_f16(tmem + (ns & 1) * 64, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
+                }
+                mma_commit(s_full + (ns & 1));
+                mma_commit(k_empty + s);
+                mbar_arrive(s_full + (ns & 1));   // publishes sinfo (release)
+                ++ns;
+                return true;
+            };
             bool ok = mbar_wait(q_full, 0, deadline, abort_flag);
-            int ns = 0, npv = 0, total = -1;
-            uint32_t idle = 0;
-            while (ok) {
-                bool progressed = false;
-                // next S: K landed and its S buffer read by the softmax two blocks back
-                if (total < 0 && ns < npv + 3) {
-                    const int s = ns % NS;
-                    if (mbar_try_wait(kfull + s, (ns / NS) & 1) &&
-                        (ns < 2 || mbar_try_wait(s_empty + (ns & 1), ((ns - 2) >> 1) & 1))) {
-                        const int j = slots[2 * s], m = slots[2 * s + 1];
-                        sinfo[2 * (ns & 3)] = j;
-                        sinfo[2 * (ns & 3) + 1] = m;
-                        if (j < 0) {
-                            total = ns;
-                            mbar_arrive(s_full + (ns & 1));
-                            mbar_arrive(s_full + (ns & 1));
-                        } else {
-                            fence_after_sync();
-                            const uint32_t ka = sbase + L::K + s * kKVBytes;
+            if (ok) ok = issue_s();
+            if (ok && total < 0) ok = issue_s();
+            for (int n = 0; ok; ++n) {
+                if (total >= 0 && n >= total) break;
+                const int sp = n % NSV;
+                ok = mbar_wait(vfull + sp, (n / NSV) & 1, deadline, abort_flag) &&
+                     mbar_wait(p_full + (n & 1), (n >> 1) & 1, deadline, abort_flag);
+                if (!ok) break;
+                fence_after_sync();
+                const uint32_t va = sbase + L::V + sp * kKVBytes;
 #pragma unroll
-                            for (int kk = 0; kk < 8; ++kk) {
-                                const uint64_t ad =
-                                    smem_desc_sw128(qa + (kk >> 2) * (kQBytes / 2) + (kk & 3) * 32, 16, 1024);
-                                const uint64_t bd =
-                                    smem_desc_sw128(ka + (kk >> 2) * (kKVBytes / 2) + (kk & 3) * 32, 16, 1024);
-                                mma_f16(tmem + (ns & 1) * 64, ad, bd, IDESC_S, kk > 0 ? 1u : 0u);
-                            }
-                            mma_commit(s_full + (ns & 1));
-                            mma_commit(k_empty + s);
-                            mbar_arrive(s_full + (ns & 1));   // publishes sinfo (release)
-                            ++ns;
-                        }
-                        progressed = true;
-                    }
+                for (int kk = 0; kk < 4; ++kk) {
+                    const uint64_t bd = smem_desc_sw128(va + kk * 2048, 8192, 1024);
+                    mma_f16_ts(tmem + 128, tmem + (n & 1) * 64 + kk * 8, bd, IDESC_PV, (n > 0 || kk > 0) ? 1u : 0u);
                 }
-                // next PV: V landed and P written
-                if (npv < ns) {
-                    const int sp = npv % NS;
-                    if (mbar_try_wait(vfull + sp, (npv / NS) & 1) && mbar_try_wait(p_full, npv & 1)) {
-                        fence_after_sync();
-                        const uint32_t va = sbase + L::V + sp * kKVBytes;
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk) {
-                            const uint64_t ad = smem_desc_sw128(pa + kk * 32, 16, 1024);
-                            const uint64_t bd = smem_desc_sw128(va + kk * 2048, 8192, 1024);
-                            mma_f16(tmem + 128, ad, bd, IDESC_PV, (npv > 0 || kk > 0) ? 1u : 0u);
-                        }
-                        mma_commit(pv_done);
-                        mma_commit(v_empty + sp);
-                        ++npv;
-                        progressed = true;
-                    }
-                }
-                if (total >= 0 && npv == total) break;
-                if (!progressed && (++idle & 63) == 0 && (*abort_flag || globaltimer() > deadline)) ok = false;
+                mma_commit(pv_done);
+                mma_commit(v_empty + sp);
+                if (total < 0) ok = issue_s();
             }
             if (!ok) {
                 *abort_flag = 1;
@@ -346,7 +335,6 @@ __global__ void __launch_bounds__(kThreads, 2)
         float m_used = -INFINITY, l = 0.f;
         int n = 0;
         bool ok = true;
-        uint8_t *prow = smem + L::P + r * 128;
         for (;;) {
             ok = __all_sync(0xffffffffu, mbar_wait(s_full + (n & 1), (n >> 1) & 1, deadline, abort_flag));
             if (!ok) break;
@@ -362,8 +350,6 @@ __global__ void __launch_bounds__(kThreads, 2)
                 tmem_ld32(lane_base + (n & 1) * 64, *reinterpret_cast<uint32_t(*)[32]>(&sr[0]));
                 tmem_ld32(lane_base + (n & 1) * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
                 tmem_wait_ld();
-                fence_before_sync();
-                mbar_arrive(s_empty + (n & 1));
                 float v[64];
                 if (sl.x == iq[hf]) {                // diagonal block: causal inside
 #pragma unroll
@@ -406,17 +392,16 @@ __global__ void __launch_bounds__(kThreads, 2)
                 const float2 s4 = fadd2(s01, s23);
                 l += s4.x + s4.y;
             } else {
-                fence_before_sync();
-                mbar_arrive(s_empty + (n & 1));
 #pragma unroll
                 for (int c = 0; c < 32; ++c) pk[c] = 0u;
             }
-            if (n > 0) {
-                ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (n - 1) & 1, deadline, abort_flag));
-                if (!ok) break;
-                fence_after_sync();
-            }
             if (__any_sync(0xffffffffu, rescale)) {
+                // O must be stable: PV_{n-1} complete
+                if (n > 0) {
+                    ok = __all_sync(0xffffffffu, mbar_wait(pv_done, (n - 1) & 1, deadline, abort_flag));
+                    if (!ok) break;
+                    fence_after_sync();
+                }
 #pragma unroll 1
                 for (int c4 = 0; c4 < 4; ++c4) {
                     uint32_t o[32];
@@ -428,15 +413,11 @@ __global__ void __launch_bounds__(kThreads, 2)
                 }
                 tmem_wait_st();
             }
-            // P row: 8 chunks of 16 B, 128-byte swizzle (chunk c at c ^ (r & 7))
-#pragma unroll
-            for (int c = 0; c < 8; ++c) {
-                uint4 w = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-                *reinterpret_cast<uint4 *>(prow + ((c ^ (r & 7)) << 4)) = w;
-            }
-            fence_proxy_async_smem();
+            // P_n (bf16 pairs) over the first 32 columns of S_n's buffer
+            tmem_st32(lane_base + (n & 1) * 64, pk);
+            tmem_wait_st();
             fence_before_sync();
-            mbar_arrive(p_full);
+            mbar_arrive(p_full + (n & 1));
             ++n;
         }
         if (ok && n > 0) {
@@ -502,7 +483,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 // Work items.  Even GQA group sizes (<= 16): per (kv head g, query block i),
 // pair the group's query heads greedily by the waste of their union (|A| +
 // |B| - 2|A n B|, smallest first, ties to the lowest pair).  One warp per
-// (g, i).  Items are ordered by query block, latest first (heavier rows early).
+// (g, i).  Items are ordered by kv head, then query block, latest first.
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_prefill_schedule_pairs(const PrefillArgs a)
 {
@@ -538,7 +519,9 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_pairs(const PrefillArg
     __syncwarp();
     if (lane == 0) {
         unsigned used = 0;
-        const int base = (nQB - 1 - i) * (a.Hq / 2) + g * (G / 2);
+        // kv-head-major: CTAs in flight share one kv head's K/V (64 MB at 128K
+        // tokens), which then stays in L2; within a head, latest blocks first
+        const int base = g * nQB * (G / 2) + (nQB - 1 - i) * (G / 2);
         for (int t = 0; t < G / 2; ++t) {
             int best = INT_MAX, ba = 0, bb = 1;
             for (int pa = 0; pa < G; ++pa) {
@@ -558,13 +541,14 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_pairs(const PrefillArg
     }
 }
 
-// Odd group sizes: adjacent query blocks (2I, 2I+1) of one head, latest first.
+// Odd group sizes: adjacent query blocks (2I, 2I+1) of one head; head-major,
+// latest blocks first.
 __global__ void k_prefill_schedule_adjacent(const PrefillArgs a)
 {
     const int nQB = (a.T + 63) >> 6, nSB = (nQB + 1) >> 1;
     const int x = blockIdx.x * blockDim.x + threadIdx.x;
     if (x >= a.Hq * nSB) return;
-    const int I = nSB - 1 - x / a.Hq, h = x % a.Hq;
+    const int h = x / nSB, I = nSB - 1 - x % nSB;   // head-major (kv heads' K/V stay in L2)
     a.items[x] = make_int4(h, 2 * I, 2 * I + 1 < nQB ? h : -1, 2 * I + 1);
 }
 
@@ -578,7 +562,7 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn()
     return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
 }
 
-constexpr int kStages = 2;
+constexpr int kKStages = 3, kVStages = 2;
 
 }  // namespace
 
@@ -617,11 +601,12 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s)
         k_prefill_schedule_adjacent<<<(a.n_items + 255) / 256, 256, 0, s>>>(a);
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
-    using L = Smem<kStages>;
+    using L = Smem<kKStages, kVStages>;
     const size_t smem = L::TOTAL;
-    e = cudaFuncSetAttribute(k_prefill_tc<kStages>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    e = cudaFuncSetAttribute(k_prefill_tc<kKStages, kVStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)smem);
     if (e != cudaSuccess) return e;
-    k_prefill_tc<kStages><<<(unsigned)a.n_items, kThreads, smem, s>>>(mq, mk, mv, a);
+    k_prefill_tc<kKStages, kVStages><<<(unsigned)a.n_items, kThreads, smem, s>>>(mq, mk, mv, a);
     return cudaGetLastError();
 }
 
