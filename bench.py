@@ -296,8 +296,11 @@ def main():
     from sparse_attention_aware_b200 import _lib
     _lib.load()
 
+    from sparse_attention_aware_b200 import parallel as PAR
     cfg = Cfg(small=args.small)
-    dec, pre, msk = build(cfg, dev)
+    # weak scaling: rank r owns shard r of a global workload (its own seeded
+    # sequences and prompt), the same per-rank size at every N
+    dec, pre, msk = build(cfg, dev, seed=1005 + 1000 * rank)
     cal_ws = sa.Workspace(dev)
     pc, pr, density = calibrate_density(pre, cal_ws, cfg.density_target)
     step = Step(cfg, dec, pre, msk, pc, pr, dev)
@@ -367,11 +370,8 @@ def main():
         parts["rbs_select"] += e[2].elapsed_time(e[3])
         parts["prefill"] += e[3].elapsed_time(e[4])
     K = args.steps
-    vals = torch.tensor([total_ms, parts["decode"], parts["masked"], parts["rbs_select"], parts["prefill"]],
-                        dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    total_ms, dec_ms, msk_ms, rbs_ms, pre_ms = [float(x) for x in vals.tolist()]
+    total_ms, dec_ms, msk_ms, rbs_ms, pre_ms = PAR.max_over_ranks(
+        [total_ms, parts["decode"], parts["masked"], parts["rbs_select"], parts["prefill"]], dev)
 
     dec_bytes = decode_group_bytes(cfg.dec)
     m = cfg.msk
@@ -527,10 +527,8 @@ def e2e(step, dec, pre, msk, cfg, args, world, dev, dist):
     torch.cuda.synchronize()
     dec_ms = sum(e[0].elapsed_time(e[1]) for e in evs)
     pre_ms = sum(e[1].elapsed_time(e[2]) for e in evs)
-    vals = torch.tensor([dec_ms, pre_ms], dtype=torch.float64, device=dev)
-    if dist is not None:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    dec_ms, pre_ms = [float(x) for x in vals.tolist()]
+    from sparse_attention_aware_b200 import parallel as PAR
+    dec_ms, pre_ms = PAR.max_over_ranks([dec_ms, pre_ms], dev)
     dec_bytes = decode_group_bytes(cfg.dec)
     csr_tiles = int(step.csr.row_ptr[-1])
     return {"value": round(world * K * dec_bytes / (dec_ms * 1e-3) / 1e9, 2), "unit": "GB/s",

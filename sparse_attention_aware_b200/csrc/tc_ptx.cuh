@@ -253,29 +253,6 @@ __device__ __forceinline__ float2 fadd2(float2 a, float2 b)
     return *reinterpret_cast<float2 *>(&d);
 }
 
-// 2^x on the FMA pipe, for a pair (takes load off the MUFU unit).  Range
-// reduction x = n + f with n = round(x) (the 1.5*2^23 add places n in the low
-// mantissa bits), 2^f for f in [-1/2, 1/2] by a cubic whose coefficients were
-// fitted here by least squares on the relative error (max relative error
-// 1.4e-4), and 2^n added into the exponent field.  x is clamped to >= -125, so
-// very negative or -inf inputs give ~2e-38 instead of 0.
-__device__ __forceinline__ float2 ex2_poly2(float2 x)
-{
-    x.x = fmaxf(x.x, -125.f);
-    x.y = fmaxf(x.y, -125.f);
-    const float2 magic = make_float2(12582912.f, 12582912.f);
-    const float2 j = fadd2(x, magic);
-    const float2 nf = fadd2(j, make_float2(-12582912.f, -12582912.f));
-    const float2 f = ffma2(nf, make_float2(-1.f, -1.f), x);
-    float2 p = ffma2(make_float2(0.055029310286045074f, 0.055029310286045074f), f,
-                     make_float2(0.24225680530071259f, 0.24225680530071259f));
-    p = ffma2(p, f, make_float2(0.6932530403137207f, 0.6932530403137207f));
-    p = ffma2(p, f, make_float2(0.9999513626098633f, 0.9999513626098633f));
-    // (bits(j) - bits(1.5*2^23)) << 23 == bits(j) << 23 (mod 2^32)
-    return make_float2(__int_as_float(__float_as_int(p.x) + (__float_as_int(j.x) << 23)),
-                       __int_as_float(__float_as_int(p.y) + (__float_as_int(j.y) << 23)));
-}
-
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi)
 {
     uint32_t r;
