@@ -6,10 +6,11 @@
 // stream).
 //
 // k_topk_score: streams the whole K context once.  One CTA = (token chunk,
-// kv head g, sequence b), 256 threads; a group of G = D/8 lanes owns one token
-// row (16 B per lane, coalesced 256 B rows at D=128) and computes the raw dot
-// product with every query head of the GQA group, so K is read once for all
-// of them.  Scores (fp32, unscaled) go to the workspace.
+// kv head g, sequence b), 256 threads.  K rows arrive in shared memory through
+// a ring of untiled bulk copies (page-row granular), and a group of G = D/8
+// lanes reads one token row from there (16 B per lane) and computes the raw
+// dot product with every query head of the GQA group, so K is read once for
+// all of them.  Scores (fp32, unscaled) go to the workspace.
 //
 // k_topk_select: one CTA of 1024 threads per (sequence, query head).  An
 // exact radix select on the order-preserving uint32 image of the fp32 score:
@@ -19,6 +20,7 @@
 // to T (ties to the lower position), in ascending position order.  Only the
 // first two passes read the whole row (see the kernel comment).
 #include "sa_internal.h"
+#include "tc_ptx.cuh"
 
 namespace sa {
 namespace {
@@ -26,108 +28,225 @@ namespace {
 constexpr int kScoreChunk = 4096;   // tokens per scoring CTA
 constexpr int kSelThreads = 1024;
 
-// Sum N = G values held by each of G lanes across the G lanes so that lane l
-// ends with the full sum of value index (l % G): at every butterfly step a lane
-// keeps the half of its values its lane bit selects and adds the partner's
-// copy of that half (G - 1 shuffles in total instead of N * log2(G)).
+// Sum G partials held by each of G lanes so that lane l ends with the total of
+// partial index l: at every butterfly step a lane keeps the lower half of its
+// positions and sends the upper half to its partner (G - 1 shuffles in all).
+// The caller stores partial p at position p ^ l (bits of l below G), which is
+// what makes "keep the lower half" right for every lane without selects: at
+// the step over lane bit o the lower half holds exactly the partials whose
+// bit o equals l's, and the partner's upper half holds the same partials.
 template <int G>
-__device__ __forceinline__ float transpose_reduce(float (&v)[G], int lane)
+__device__ __forceinline__ float transpose_reduce(float (&v)[G])
 {
 #pragma unroll
-    for (int o = G / 2, cnt = G / 2; o >= 1; o >>= 1, cnt >>= 1) {
-        const bool upper = lane & o;
+    for (int cnt = G / 2; cnt >= 1; cnt >>= 1) {
 #pragma unroll
-        for (int i = 0; i < cnt; ++i) {
-            const float send = upper ? v[i] : v[i + cnt];
-            const float keep = upper ? v[i + cnt] : v[i];
-            v[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
-        }
+        for (int i = 0; i < cnt; ++i) v[i] += __shfl_xor_sync(0xffffffffu, v[i + cnt], cnt);
     }
     return v[0];
 }
 
-// One group of G = D/8 lanes owns U = G/HPG consecutive token rows per step;
-// the G partial sums (U rows x HPG heads) are reduced with transpose_reduce,
-// after which lane gl holds row gl / HPG, head gl % HPG.
+// Tile geometry of the scoring kernel.  One group of G = D/8 lanes owns U =
+// G/HPG consecutive token rows per step (STEP rows per CTA step); a ring stage
+// holds TT >= 64 tokens (R steps) of one kv head's K rows.
+template <int D, int HPG>
+struct ScoreGeom {
+    static constexpr int G = D / 8, GPW = 32 / G, NG = 8 * GPW, U = G / HPG;
+    static constexpr int STEP = NG * U;
+    static constexpr int TT = STEP >= 64 ? STEP : 64;
+    static constexpr int R = TT / STEP;
+    static constexpr int STAGE = TT * D * 2;
+    static constexpr int NS0 = (64 * 1024) / STAGE;   // 3 CTAs per SM at D=128
+    static constexpr int NS = NS0 < 2 ? 2 : (NS0 > 8 ? 8 : NS0);
+    static constexpr int MAXJ = (TT + 31) / 32;   // page spans per lane of the producer warp
+    static constexpr int SMEM = NS * STAGE + 2 * NS * 8 + NS * 8 * 4 + 16;
+    static constexpr int THREADS = 8 * 32 + 32;    // 8 consumer warps + 1 producer warp
+};
+
+constexpr uint64_t kScoreWaitNs = 1000ull * 1000 * 1000;   // 1 s
+
+// The K rows of a CTA's token chunk stream through an NS-stage shared-memory
+// ring filled by untiled bulk copies (one per page span of a tile: whole page
+// rows when P <= TT, else a TT-token piece of one).  Warp 8 is the producer:
+// it refills a stage once all 8 consumer warps have released it (per-stage
+// "empty" mbarriers, so consumer warps drift freely within the ring) and keeps
+// the page-table entries of the next tile in registers.  Rows whose page
+// entry is out of range are recorded as a device fault and score -inf, so they
+// are never selected.
 template <int D, int HPG, bool QF32>
-__global__ void __launch_bounds__(256) k_topk_score(const TopkArgs a)
+__global__ void __launch_bounds__(ScoreGeom<D, HPG>::THREADS) k_topk_score(const TopkArgs a)
 {
-    constexpr int G = D / 8, GPW = 32 / G, NG = 8 * GPW;
-    constexpr int U = G / HPG;
-    static_assert(U >= 1 && U * HPG == G, "rows per step");
+    using Gm = ScoreGeom<D, HPG>;
+    constexpr int G = Gm::G, GPW = Gm::GPW, U = Gm::U, TT = Gm::TT, NS = Gm::NS, MAXJ = Gm::MAXJ;
+    constexpr int HL = HPG == 1 ? 0 : HPG == 2 ? 1 : HPG == 4 ? 2 : 3;   // log2(HPG)
+    extern __shared__ __align__(128) uint8_t sm[];
+    uint64_t *full = reinterpret_cast<uint64_t *>(sm + NS * Gm::STAGE);
+    uint64_t *empty = full + NS;
+    uint32_t *badm = reinterpret_cast<uint32_t *>(empty + NS);   // [NS][8] bad-span bits
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(badm + NS * 8);
+
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    const int gl = lane & (G - 1), sub = lane / G;
     const int chunk = blockIdx.x, g = blockIdx.y, b = blockIdx.z;
     const int Lcap = a.c.max_pages << a.c.Plog2;
     int L = __ldg(a.c.sl + b);
     if (L < 0 || L > Lcap) {
-        fault(a.st, CHK_SEQ_LEN, L);
+        if (threadIdx.x == 0 && chunk == 0 && g == 0) fault(a.st, CHK_SEQ_LEN, L);
         L = L < 0 ? 0 : Lcap;
     }
     const int t0 = chunk * kScoreChunk;
     const int t1 = min(t0 + kScoreChunk, L);
     if (t0 >= t1) return;
+    const int ntiles = (t1 - t0 + TT - 1) / TT;
+    // page spans: SPAN = min(P, TT) tokens, nsp = TT / SPAN per tile
+    constexpr int TL = TT == 64 ? 6 : TT == 128 ? 7 : 8;   // log2(TT)
+    static_assert((1 << TL) == TT, "tile size");
+    const int slog2 = min(a.c.Plog2, TL);
+    const int SPAN = 1 << slog2;
+    const int nsp = TT >> slog2;
 
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < NS; ++s) {
+            tc::mbar_init(full + s, 1);
+            tc::mbar_init(empty + s, 8);
+        }
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+    __syncthreads();
+    const uint64_t deadline = tc::globaltimer() + kScoreWaitNs;
+
+    if (warp == 8) {
+        // ---------------------------------------------------------------- producer
+        const int32_t *ptb = a.c.pt + (size_t)b * a.c.max_pages;
+        const int Pm = (1 << a.c.Plog2) - 1;
+        int pg[MAXJ];
+        auto fetch = [&](int tile) {
+#pragma unroll
+            for (int j = 0; j < MAXJ; ++j) {
+                const int sp = lane + 32 * j;
+                const int ts = t0 + tile * TT + (sp << slog2);
+                pg[j] = (tile < ntiles && sp < nsp && ts < t1) ? __ldg(ptb + (ts >> a.c.Plog2)) : -1;
+            }
+        };
+        fetch(0);
+        int issued = 0;
+        for (int i = 0; i < ntiles; ++i) {
+            const int s = i % NS;
+            if (i >= NS) {
+                const bool ok = __all_sync(
+                    0xffffffffu, tc::mbar_wait(empty + s, (uint32_t)((i / NS) - 1) & 1u, deadline, abort_flag));
+                if (!ok) break;
+            }
+            uint8_t *dst = sm + s * Gm::STAGE;
+            uint32_t bytes = 0;
+            bool go[MAXJ];
+#pragma unroll
+            for (int j = 0; j < MAXJ; ++j) {
+                const int sp = lane + 32 * j;
+                const int ts = t0 + i * TT + (sp << slog2);
+                const bool need = sp < nsp && ts < t1;
+                const bool bad = need && (pg[j] < 0 || pg[j] >= a.c.num_pages);
+                if (bad) fault(a.st, CHK_PAGE, pg[j]);
+                go[j] = need && !bad;
+                if (go[j]) bytes += (uint32_t)SPAN * D * 2;
+                const unsigned bw = __ballot_sync(0xffffffffu, bad);
+                if (lane == 0) badm[s * 8 + j] = bw;
+            }
+#pragma unroll
+            for (int o = 16; o >= 1; o >>= 1) bytes += __shfl_xor_sync(0xffffffffu, bytes, o);
+            if (lane == 0) tc::mbar_arrive_expect_tx(full + s, bytes);
+            __syncwarp();
+#pragma unroll
+            for (int j = 0; j < MAXJ; ++j) {
+                if (!go[j]) continue;
+                const int sp = lane + 32 * j;
+                const int ts = t0 + i * TT + (sp << slog2);
+                const uint16_t *src =
+                    a.c.k + ((((size_t)pg[j] * a.c.Hkv + g) << a.c.Plog2) + (ts & Pm)) * D;
+                tc::bulk_load(dst + ((size_t)sp << slog2) * D * 2, src, (uint32_t)SPAN * D * 2, full + s);
+            }
+            issued = i + 1;
+            fetch(i + 1);
+        }
+        if (issued < ntiles) {
+            // the consumers stopped releasing stages: record it and wait
+            // (bounded) for the copies still in flight before the CTA's shared
+            // memory is released
+            *abort_flag = 1;
+            if (lane == 0) {
+                fault(a.st, CHK_WAIT, issued);
+                const uint64_t dl = tc::globaltimer() + kScoreWaitNs;
+                volatile int zero = 0;
+                for (int j = max(0, issued - NS); j < issued; ++j)
+                    tc::mbar_wait(full + j % NS, (uint32_t)(j / NS) & 1u, dl, &zero);
+            }
+        }
+        return;
+    }
+
+    // -------------------------------------------------------------------- consumers
+    const int gl = lane & (G - 1), sub = lane / G;
+    // partial p = (row u, head j) = u * HPG + j lives at position p ^ gl, so the
+    // lane reads its rows in the order u ^ (gl >> HL) and holds its query heads
+    // in the order j ^ (gl & (HPG - 1))
+    const int ux = gl >> HL, jx = gl & (HPG - 1);
     float qv[HPG][8];
 #pragma unroll
-    for (int j = 0; j < HPG; ++j) {
-        const size_t row = (size_t)b * a.Hq + g * HPG + j;
+    for (int jj = 0; jj < HPG; ++jj) {
+        const size_t row = (size_t)b * a.Hq + g * HPG + (jj ^ jx);
         if (QF32) {
             const float4 *qp = reinterpret_cast<const float4 *>(reinterpret_cast<const float *>(a.q) +
                                                                 row * D + gl * 8);
             float4 x0 = __ldg(qp), x1 = __ldg(qp + 1);
-            qv[j][0] = x0.x; qv[j][1] = x0.y; qv[j][2] = x0.z; qv[j][3] = x0.w;
-            qv[j][4] = x1.x; qv[j][5] = x1.y; qv[j][6] = x1.z; qv[j][7] = x1.w;
+            qv[jj][0] = x0.x; qv[jj][1] = x0.y; qv[jj][2] = x0.z; qv[jj][3] = x0.w;
+            qv[jj][4] = x1.x; qv[jj][5] = x1.y; qv[jj][6] = x1.z; qv[jj][7] = x1.w;
         } else {
             uint4 w = ldg_nc_v4(reinterpret_cast<const uint16_t *>(a.q) + row * D + gl * 8);
-            qv[j][0] = bf_lo(w.x); qv[j][1] = bf_hi(w.x); qv[j][2] = bf_lo(w.y); qv[j][3] = bf_hi(w.y);
-            qv[j][4] = bf_lo(w.z); qv[j][5] = bf_hi(w.z); qv[j][6] = bf_lo(w.w); qv[j][7] = bf_hi(w.w);
+            qv[jj][0] = bf_lo(w.x); qv[jj][1] = bf_hi(w.x); qv[jj][2] = bf_lo(w.y); qv[jj][3] = bf_hi(w.y);
+            qv[jj][4] = bf_lo(w.z); qv[jj][5] = bf_hi(w.z); qv[jj][6] = bf_lo(w.w); qv[jj][7] = bf_hi(w.w);
         }
     }
-    const int32_t *ptb = a.c.pt + (size_t)b * a.c.max_pages;
-    const int Pm = (1 << a.c.Plog2) - 1;
-    float *srow = a.scores + ((size_t)b * a.Hq + g * HPG) * a.Lcap;
-    const int my_u = gl / HPG, my_j = gl % HPG;
+    // after the reduction lane gl holds partial gl: row gl >> HL, head gl & (HPG-1)
+    float *sout = a.scores + ((size_t)b * a.Hq + g * HPG + (gl & (HPG - 1))) * a.Lcap;
+    const int my_u = gl >> HL;
 
-    for (int base0 = t0 + warp * GPW * U; base0 < t1; base0 += NG * U) {
-        const int base = base0 + sub * U;
-        uint4 kr[U];
-        bool ok[U];
+    for (int i = 0; i < ntiles; ++i) {
+        const int s = i % NS;
+        const bool ok = __all_sync(0xffffffffu,
+                                   tc::mbar_wait(full + s, (uint32_t)(i / NS) & 1u, deadline, abort_flag));
+        if (!ok) {
+            // a copy never completed: record it and stop this warp
+            *abort_flag = 1;
+            if (lane == 0) fault(a.st, CHK_WAIT, i);
+            break;
+        }
+        const uint8_t *stage = sm + s * Gm::STAGE + gl * 16;
+        const int tb = t0 + i * TT;
 #pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int t = base + u;
-            ok[u] = t < t1;
-            int page = 0;
-            if (ok[u]) {
-                page = __ldg(ptb + (t >> a.c.Plog2));
-                if (page < 0 || page >= a.c.num_pages) {
-                    fault(a.st, CHK_PAGE, page);
-                    ok[u] = false;
+        for (int st = 0; st < Gm::R; ++st) {
+            const int r0 = st * Gm::STEP + (warp * GPW + sub) * U;   // first row of this group
+            float part[G];
+#pragma unroll
+            for (int uu = 0; uu < U; ++uu) {
+                const uint4 kr = *reinterpret_cast<const uint4 *>(stage + (size_t)(r0 + (uu ^ ux)) * D * 2);
+                const float kf[8] = {bf_lo(kr.x), bf_hi(kr.x), bf_lo(kr.y), bf_hi(kr.y),
+                                     bf_lo(kr.z), bf_hi(kr.z), bf_lo(kr.w), bf_hi(kr.w)};
+#pragma unroll
+                for (int jj = 0; jj < HPG; ++jj) {
+                    float p = qv[jj][0] * kf[0];
+#pragma unroll
+                    for (int e = 1; e < 8; ++e) p = fmaf(qv[jj][e], kf[e], p);
+                    part[uu * HPG + jj] = p;
                 }
             }
-            const size_t off = ((((size_t)page * a.c.Hkv + g) << a.c.Plog2) + (t & Pm)) * D + gl * 8;
-            kr[u] = ok[u] ? ldg_nc_v4(a.c.k + off) : make_uint4(0, 0, 0, 0);
+            const float sc = transpose_reduce<G>(part);
+            const int r = r0 + my_u;
+            const int sp = r >> slog2;
+            const bool bad = (badm[s * 8 + (sp >> 5)] >> (sp & 31)) & 1u;
+            if (tb + r < t1) sout[tb + r] = bad ? -INFINITY : sc;
         }
-        float part[G];
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const float kf[8] = {bf_lo(kr[u].x), bf_hi(kr[u].x), bf_lo(kr[u].y), bf_hi(kr[u].y),
-                                 bf_lo(kr[u].z), bf_hi(kr[u].z), bf_lo(kr[u].w), bf_hi(kr[u].w)};
-#pragma unroll
-            for (int j = 0; j < HPG; ++j) {
-                float p = qv[j][0] * kf[0];
-#pragma unroll
-                for (int e = 1; e < 8; ++e) p = fmaf(qv[j][e], kf[e], p);
-                part[u * HPG + j] = p;
-            }
-        }
-        const float sc = transpose_reduce<G>(part, gl);
-        const int t = base + my_u;
-        bool okm = false;
-#pragma unroll
-        for (int u = 0; u < U; ++u) okm = (u == my_u) ? ok[u] : okm;
-        // an unreadable row (bad page) scores -inf so it is never selected
-        if (t < t1) srow[(size_t)my_j * a.Lcap + t] = okm ? sc : -INFINITY;
+        __syncwarp();
+        if (lane == 0) tc::mbar_arrive(empty + s);
     }
 }
 
@@ -164,7 +283,9 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total)
 // One radix digit pass over the elements whose key matches (prefix, pmask):
 // histogram of the digit at `shift` (nbits wide), then the digit D holding the
 // need-th largest element; `need` drops by the count above D.
-template <typename KeyAt>
+// BATCH keys per thread are loaded before any is counted, so that many loads
+// are in flight.
+template <int BATCH, typename KeyAt>
 __device__ void digit_pass(KeyAt key_at, int n, int shift, int nbits, uint32_t &prefix, uint32_t &pmask,
                            unsigned &need, unsigned *hist, int *warp_tot, unsigned &s_digit, unsigned &s_above)
 {
@@ -172,9 +293,19 @@ __device__ void digit_pass(KeyAt key_at, int n, int shift, int nbits, uint32_t &
     const int nb = 1 << nbits;
     for (int i = tid; i < nb; i += kSelThreads) hist[i] = 0;
     __syncthreads();
-    for (int t = tid; t < n; t += kSelThreads) {
-        const uint32_t key = key_at(t);
-        if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+    for (int t0 = 0; t0 < n; t0 += kSelThreads * BATCH) {
+        uint32_t kk[BATCH];
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+            const int t = t0 + u * kSelThreads + tid;
+            kk[u] = t < n ? key_at(t) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+            const int t = t0 + u * kSelThreads + tid;
+            const bool act = t < n && (kk[u] & pmask) == prefix;
+            if (act) atomicAdd(&hist[(kk[u] >> shift) & (nb - 1)], 1u);
+        }
     }
     __syncthreads();
     // thread i owns bins in descending order [nb - (i+1)*per, nb - i*per)
@@ -245,31 +376,42 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const TopkArgs a)
 
     uint32_t prefix = 0, pmask = 0;
     unsigned need = (unsigned)k;
-    digit_pass(full_key, L, 21, 11, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
+    digit_pass<8>(full_key, L, 21, 11, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
     const uint32_t D1 = prefix >> 21;
 
     // pass 2: bitmap of top digit > D1, candidates with top digit == D1
     if (tid == 0) s_ncand = 0;
     __syncthreads();
-    for (int w0 = warp * 32; w0 < nw * 32; w0 += kSelThreads) {
-        const int t = w0 + lane;
-        const uint32_t key = t < L ? full_key(t) : 0u;
-        const uint32_t dg = key >> 21;
-        const unsigned hi = __ballot_sync(0xffffffffu, t < L && dg > D1);
-        const unsigned eq = __ballot_sync(0xffffffffu, t < L && dg == D1);
-        if (lane == 0) {
-            above[w0 >> 5] = hi;
-            eqmap[w0 >> 5] = 0u;
+    for (int wb = warp * 32; wb < nw * 32; wb += kSelThreads * 8) {
+        uint32_t kk[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int t = wb + u * kSelThreads + lane;
+            kk[u] = t < L ? full_key(t) : 0u;
         }
-        if (eq) {
-            unsigned base = 0;
-            if (lane == 0) base = atomicAdd(&s_ncand, (unsigned)__popc(eq));
-            base = __shfl_sync(0xffffffffu, base, 0);
-            if (eq >> lane & 1) {
-                const unsigned slot = base + __popc(eq & ((1u << lane) - 1u));
-                if (slot < kCandCap) {
-                    ckey[slot] = key;
-                    cpos[slot] = (uint32_t)t;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int w0 = wb + u * kSelThreads;
+            if (w0 >= nw * 32) break;
+            const int t = w0 + lane;
+            const uint32_t key = kk[u];
+            const uint32_t dg = key >> 21;
+            const unsigned hi = __ballot_sync(0xffffffffu, t < L && dg > D1);
+            const unsigned eq = __ballot_sync(0xffffffffu, t < L && dg == D1);
+            if (lane == 0) {
+                above[w0 >> 5] = hi;
+                eqmap[w0 >> 5] = 0u;
+            }
+            if (eq) {
+                unsigned base = 0;
+                if (lane == 0) base = atomicAdd(&s_ncand, (unsigned)__popc(eq));
+                base = __shfl_sync(0xffffffffu, base, 0);
+                if (eq >> lane & 1) {
+                    const unsigned slot = base + __popc(eq & ((1u << lane) - 1u));
+                    if (slot < kCandCap) {
+                        ckey[slot] = key;
+                        cpos[slot] = (uint32_t)t;
+                    }
                 }
             }
         }
@@ -279,8 +421,8 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const TopkArgs a)
     int written = 0;
     if (ncand <= kCandCap) {
         auto cand_key = [&](int i) { return ckey[i]; };
-        digit_pass(cand_key, (int)ncand, 10, 11, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
-        digit_pass(cand_key, (int)ncand, 0, 10, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
+        digit_pass<2>(cand_key, (int)ncand, 10, 11, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
+        digit_pass<2>(cand_key, (int)ncand, 0, 10, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
         const uint32_t T = prefix;   // the k-th largest key; take `need` elements equal to T
         for (int i = tid; i < (int)ncand; i += kSelThreads) {
             const uint32_t key = ckey[i], t = cpos[i];
@@ -320,8 +462,8 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const TopkArgs a)
         written = sel_tot;
     } else {
         // candidate overflow (many equal or clustered scores): full-row passes
-        digit_pass(full_key, L, 10, 11, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
-        digit_pass(full_key, L, 0, 10, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
+        digit_pass<8>(full_key, L, 10, 11, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
+        digit_pass<8>(full_key, L, 0, 10, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
         const uint32_t T = prefix;
         int eq_seen = 0;
 #pragma unroll 1
@@ -349,7 +491,11 @@ cudaError_t launch_score(const TopkArgs &a, cudaStream_t s)
 {
     const int Lcap = a.c.max_pages << a.c.Plog2;
     dim3 grid((Lcap + kScoreChunk - 1) / kScoreChunk, a.c.Hkv, a.c.B);
-    k_topk_score<D, HPG, QF32><<<grid, 256, 0, s>>>(a);
+    constexpr int smem = ScoreGeom<D, HPG>::SMEM;
+    cudaError_t e = cudaFuncSetAttribute(k_topk_score<D, HPG, QF32>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    k_topk_score<D, HPG, QF32><<<grid, ScoreGeom<D, HPG>::THREADS, smem, s>>>(a);
     return cudaGetLastError();
 }
 

@@ -99,6 +99,11 @@ def test_bad_device_data_is_recorded_not_faulted(cuda_dev):
     (128, 64, 8, 1, 100, torch.bfloat16),
     (64, 16, 4, 4, 33, torch.float32),
     (128, 16, 16, 2, 512, torch.bfloat16),
+    # 8 query heads per kv head (two compute steps per ring tile), one query
+    # head per kv head (256-token tiles of four 64-token pages)
+    (128, 16, 8, 1, 50, torch.bfloat16),
+    (64, 64, 8, 1, 40, torch.float32),
+    (128, 64, 2, 2, 70, torch.bfloat16),
 ])
 def test_topk_bit_exact_random(cuda_dev, d, P, Hq, Hkv, k, qdt):
     lens = [5, k, k + 1, 3000, 4100]
@@ -112,6 +117,20 @@ def test_topk_bit_exact_random(cuda_dev, d, P, Hq, Hkv, k, qdt):
     ws.raise_on_fault()
     np.testing.assert_array_equal(sel.count.cpu().numpy(), ref_cnt)
     np.testing.assert_array_equal(sel.idx.cpu().numpy(), ref_idx)
+
+
+def test_topk_bad_page_is_recorded_and_never_selected(cuda_dev):
+    cache, q = W.random_decode(8, 2, 4, 2, 128, [300, 200], 16)
+    pt = cache.page_table.clone()
+    pt[0, 2] = 10 ** 6                      # tokens 32..47 of sequence 0
+    bad = W.PagedCache(cache.k, cache.v, pt, cache.seq_lens).to(cuda_dev)
+    ws = sa.Workspace(cuda_dev)
+    sel = sa.select_topk(bad, q.to(cuda_dev), 40, ws=ws)
+    st, det = ws.status()
+    assert st == 5 and det[1] == 2           # SA_ERR_DEVICE_FAULT, page check
+    idx = sel.idx.cpu().numpy()
+    assert (sel.count.cpu().numpy() == 40).all()
+    assert not np.isin(idx[0], np.arange(32, 48)).any()
 
 
 def test_topk_ties_go_to_lower_position(cuda_dev):
