@@ -283,31 +283,14 @@ __device__ __forceinline__ int block_excl_scan(int v, int *warp_tot, int &total)
 // One radix digit pass over the elements whose key matches (prefix, pmask):
 // histogram of the digit at `shift` (nbits wide), then the digit D holding the
 // need-th largest element; `need` drops by the count above D.
-// BATCH keys per thread are loaded before any is counted, so that many loads
-// are in flight.
-template <int BATCH, typename KeyAt>
-__device__ void digit_pass(KeyAt key_at, int n, int shift, int nbits, uint32_t &prefix, uint32_t &pmask,
-                           unsigned &need, unsigned *hist, int *warp_tot, unsigned &s_digit, unsigned &s_above)
+// Digit selection after a histogram pass: the digit D holding the need-th
+// largest element among those matching (prefix, pmask); `need` drops by the
+// count above D and D is appended to the prefix.
+__device__ void pick_digit(int shift, int nbits, uint32_t &prefix, uint32_t &pmask, unsigned &need,
+                           unsigned *hist, int *warp_tot, unsigned &s_digit, unsigned &s_above)
 {
     const int tid = threadIdx.x;
     const int nb = 1 << nbits;
-    for (int i = tid; i < nb; i += kSelThreads) hist[i] = 0;
-    __syncthreads();
-    for (int t0 = 0; t0 < n; t0 += kSelThreads * BATCH) {
-        uint32_t kk[BATCH];
-#pragma unroll
-        for (int u = 0; u < BATCH; ++u) {
-            const int t = t0 + u * kSelThreads + tid;
-            kk[u] = t < n ? key_at(t) : 0u;
-        }
-#pragma unroll
-        for (int u = 0; u < BATCH; ++u) {
-            const int t = t0 + u * kSelThreads + tid;
-            const bool act = t < n && (kk[u] & pmask) == prefix;
-            if (act) atomicAdd(&hist[(kk[u] >> shift) & (nb - 1)], 1u);
-        }
-    }
-    __syncthreads();
     // thread i owns bins in descending order [nb - (i+1)*per, nb - i*per)
     const int per = nb / kSelThreads;
     int mine = 0;
@@ -334,6 +317,34 @@ __device__ void digit_pass(KeyAt key_at, int n, int shift, int nbits, uint32_t &
     __syncthreads();
 }
 
+// BATCH keys per thread are loaded before any is counted, so that many loads
+// are in flight.
+template <int BATCH, typename KeyAt>
+__device__ void digit_pass(KeyAt key_at, int n, int shift, int nbits, uint32_t &prefix, uint32_t &pmask,
+                           unsigned &need, unsigned *hist, int *warp_tot, unsigned &s_digit, unsigned &s_above)
+{
+    const int tid = threadIdx.x;
+    const int nb = 1 << nbits;
+    for (int i = tid; i < nb; i += kSelThreads) hist[i] = 0;
+    __syncthreads();
+    for (int t0 = 0; t0 < n; t0 += kSelThreads * BATCH) {
+        uint32_t kk[BATCH];
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+            const int t = t0 + u * kSelThreads + tid;
+            kk[u] = t < n ? key_at(t) : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < BATCH; ++u) {
+            const int t = t0 + u * kSelThreads + tid;
+            const bool act = t < n && (kk[u] & pmask) == prefix;
+            if (act) atomicAdd(&hist[(kk[u] >> shift) & (nb - 1)], 1u);
+        }
+    }
+    __syncthreads();
+    pick_digit(shift, nbits, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
+}
+
 constexpr int kCandCap = 4096;
 
 // Exact top-k of one (sequence, query head) score row.  Pass 1 histograms the
@@ -345,7 +356,7 @@ constexpr int kCandCap = 4096;
 // position order from the bitmaps.  If the candidates overflow their buffer,
 // the remaining digit passes and the emission read the full row instead.
 // Dynamic shared memory: 2 bitmaps of Lcap bits + 2 x kCandCap words.
-__global__ void __launch_bounds__(kSelThreads) k_topk_select(const TopkArgs a)
+__global__ void __launch_bounds__(kSelThreads, 2) k_topk_select(const TopkArgs a)
 {
     extern __shared__ uint32_t dsm[];
     __shared__ unsigned hist[2048];
@@ -354,7 +365,7 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const TopkArgs a)
 
     const int row = blockIdx.x;
     const int b = row / a.Hq;
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int Lcap = a.c.max_pages << a.c.Plog2;
     int L = __ldg(a.c.sl + b);
     if (L < 0 || L > Lcap) L = L < 0 ? 0 : Lcap;   // recorded by the scoring kernel
@@ -374,43 +385,87 @@ __global__ void __launch_bounds__(kSelThreads) k_topk_select(const TopkArgs a)
     uint32_t *cpos = ckey + kCandCap;
     auto full_key = [&](int t) { return f2key(__ldcg(sc + t)); };
 
-    uint32_t prefix = 0, pmask = 0;
-    unsigned need = (unsigned)k;
-    digit_pass<8>(full_key, L, 21, 11, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
-    const uint32_t D1 = prefix >> 21;
-
-    // pass 2: bitmap of top digit > D1, candidates with top digit == D1
-    if (tid == 0) s_ncand = 0;
+    // pass 1: histogram of the top 11 key bits over the whole row, 16-byte
+    // loads (the row buffer holds a multiple of 16 entries, so the last vector
+    // is readable; entries at or past L are not counted)
+    const float4 *row4 = reinterpret_cast<const float4 *>(sc);
+    const int nv = (L + 3) >> 2;
+    for (int i = tid; i < 2048; i += kSelThreads) hist[i] = 0;
     __syncthreads();
-    for (int wb = warp * 32; wb < nw * 32; wb += kSelThreads * 8) {
-        uint32_t kk[8];
+    for (int v0 = 0; v0 < nv; v0 += kSelThreads * 4) {
+        float4 x[4];
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int t = wb + u * kSelThreads + lane;
-            kk[u] = t < L ? full_key(t) : 0u;
+        for (int u = 0; u < 4; ++u) {
+            const int v = v0 + u * kSelThreads + tid;
+            x[u] = v < nv ? __ldcg(row4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
         }
 #pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int w0 = wb + u * kSelThreads;
-            if (w0 >= nw * 32) break;
-            const int t = w0 + lane;
-            const uint32_t key = kk[u];
-            const uint32_t dg = key >> 21;
-            const unsigned hi = __ballot_sync(0xffffffffu, t < L && dg > D1);
-            const unsigned eq = __ballot_sync(0xffffffffu, t < L && dg == D1);
-            if (lane == 0) {
-                above[w0 >> 5] = hi;
-                eqmap[w0 >> 5] = 0u;
+        for (int u = 0; u < 4; ++u) {
+            const int t = (v0 + u * kSelThreads + tid) * 4;
+            if (t + 3 < L) {
+                atomicAdd(&hist[f2key(x[u].x) >> 21], 1u);
+                atomicAdd(&hist[f2key(x[u].y) >> 21], 1u);
+                atomicAdd(&hist[f2key(x[u].z) >> 21], 1u);
+                atomicAdd(&hist[f2key(x[u].w) >> 21], 1u);
+            } else if (t < L) {
+                atomicAdd(&hist[f2key(x[u].x) >> 21], 1u);
+                if (t + 1 < L) atomicAdd(&hist[f2key(x[u].y) >> 21], 1u);
+                if (t + 2 < L) atomicAdd(&hist[f2key(x[u].z) >> 21], 1u);
             }
-            if (eq) {
-                unsigned base = 0;
-                if (lane == 0) base = atomicAdd(&s_ncand, (unsigned)__popc(eq));
-                base = __shfl_sync(0xffffffffu, base, 0);
-                if (eq >> lane & 1) {
-                    const unsigned slot = base + __popc(eq & ((1u << lane) - 1u));
-                    if (slot < kCandCap) {
-                        ckey[slot] = key;
-                        cpos[slot] = (uint32_t)t;
+        }
+    }
+    __syncthreads();
+    uint32_t prefix = 0, pmask = 0;
+    unsigned need = (unsigned)k;
+    pick_digit(21, 11, prefix, pmask, need, hist, warp_tot, s_digit, s_above);
+    const uint32_t D1 = prefix >> 21;
+
+    // pass 2: bitmap of top digit > D1, candidates with top digit == D1.  A
+    // lane holds 4 consecutive entries, so 8 lanes make one 32-bit bitmap
+    // word: each lane's 4-bit nibble is shifted into place and OR-ed across
+    // the 8 lanes with xor shuffles.
+    if (tid == 0) s_ncand = 0;
+    __syncthreads();
+    for (int v0 = 0; v0 < nv; v0 += kSelThreads * 4) {
+        float4 x[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int v = v0 + u * kSelThreads + tid;
+            x[u] = v < nv ? __ldcg(row4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int v = v0 + u * kSelThreads + tid;
+            const int t = v * 4;
+            const uint32_t kk[4] = {f2key(x[u].x), f2key(x[u].y), f2key(x[u].z), f2key(x[u].w)};
+            uint32_t hn = 0, en = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const bool in = t + j < L;
+                const uint32_t dg = kk[j] >> 21;
+                hn |= (uint32_t)(in && dg > D1) << j;
+                en |= (uint32_t)(in && dg == D1) << j;
+            }
+            uint32_t hw = hn << (4 * (lane & 7)), ew = en << (4 * (lane & 7));
+#pragma unroll
+            for (int o = 1; o < 8; o <<= 1) {
+                hw |= __shfl_xor_sync(0xffffffffu, hw, o);
+                ew |= __shfl_xor_sync(0xffffffffu, ew, o);
+            }
+            if ((lane & 7) == 0 && (v >> 3) < nw) {
+                above[v >> 3] = hw;
+                eqmap[v >> 3] = 0u;
+            }
+            if (en) {
+                unsigned slot = atomicAdd(&s_ncand, (unsigned)__popc(en));
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    if (en >> j & 1) {
+                        if (slot < kCandCap) {
+                            ckey[slot] = kk[j];
+                            cpos[slot] = (uint32_t)(t + j);
+                        }
+                        ++slot;
                     }
                 }
             }
