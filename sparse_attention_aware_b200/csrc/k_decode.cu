@@ -45,6 +45,8 @@ __device__ __forceinline__ int locate_entry(const int4 *ent, int ne, int pos)
 template <int D, bool QF32, bool BLOCKS, int U>
 __global__ void __launch_bounds__(256) k_decode_split(const DecodeArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     using C = DecodeCfg<D>;
     constexpr int G = C::G, GPW = C::GPW, NG = C::NG;
     __shared__ float s_m[NG], s_l[NG];
@@ -248,6 +250,8 @@ __global__ void __launch_bounds__(D) k_decode_combine(const float *__restrict__ 
                                                        uint16_t *__restrict__ out,
                                                        float *__restrict__ lse)
 {
+    pdl_wait();
+    pdl_trigger();
     const int row = blockIdx.x, c = threadIdx.x;
     const float *ml = part_ml + (size_t)row * S * 2;
     float M = -INFINITY;
@@ -272,7 +276,7 @@ template <int D, bool QF32, bool BLOCKS>
 cudaError_t launch_split(const DecodeArgs &a, cudaStream_t s)
 {
     dim3 grid(a.S, a.Hq, a.c.B);
-    k_decode_split<D, QF32, BLOCKS, 4><<<grid, 256, 0, s>>>(a);
+    if (cudaError_t e_ = launch_pdl(k_decode_split<D, QF32, BLOCKS, 4>, dim3(grid), dim3(256), 0, s, a)) return e_;
     return cudaGetLastError();
 }
 
@@ -280,12 +284,14 @@ template <int D>
 cudaError_t launch_d(const DecodeArgs &a, cudaStream_t s)
 {
     cudaError_t e;
-    if (a.blocks)
+    if (decode_gqa_supported(a))
+        e = launch_decode_gqa_split(a, s);
+    else if (a.blocks)
         e = a.q_f32 ? launch_split<D, true, true>(a, s) : launch_split<D, false, true>(a, s);
     else
         e = a.q_f32 ? launch_split<D, true, false>(a, s) : launch_split<D, false, false>(a, s);
     if (e != cudaSuccess) return e;
-    k_decode_combine<D><<<a.c.B * a.Hq, D, 0, s>>>(a.part_o, a.part_ml, a.S, a.out, a.lse);
+    if (cudaError_t e_ = launch_pdl(k_decode_combine<D>, dim3(a.c.B * a.Hq), dim3(D), 0, s, a.part_o, a.part_ml, a.S, a.out, a.lse)) return e_;
     return cudaGetLastError();
 }
 

@@ -136,6 +136,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     k_prefill_tc(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                  const __grid_constant__ CUtensorMap tmV, const PrefillArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     using L = Smem<NSK, NSV>;
     extern __shared__ __align__(1024) uint8_t smem[];
     const uint32_t sbase = smem_u32(smem);
@@ -487,6 +489,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_prefill_schedule_pairs(const PrefillArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int cost[8][kMaxPairGroup][kMaxPairGroup];
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int nQB = (a.T + 63) >> 6;
@@ -545,6 +549,8 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_pairs(const PrefillArg
 // latest blocks first.
 __global__ void k_prefill_schedule_adjacent(const PrefillArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     const int nQB = (a.T + 63) >> 6, nSB = (nQB + 1) >> 1;
     const int x = blockIdx.x * blockDim.x + threadIdx.x;
     if (x >= a.Hq * nSB) return;
@@ -595,10 +601,13 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s)
     const int nQB = (a.T + 63) / 64;
     const int G = a.Hq / a.c.Hkv;
     if (a.n_items <= 0) return cudaSuccess;
-    if (G % 2 == 0 && G <= kMaxPairGroup)
-        k_prefill_schedule_pairs<<<(a.c.Hkv * nQB + 7) / 8, 256, 0, s>>>(a);
-    else
-        k_prefill_schedule_adjacent<<<(a.n_items + 255) / 256, 256, 0, s>>>(a);
+    if (G % 2 == 0 && G <= kMaxPairGroup) {
+        if (cudaError_t e_ = launch_pdl(k_prefill_schedule_pairs, dim3((a.c.Hkv * nQB + 7) / 8), dim3(256), 0, s, a))
+            return e_;
+    } else {
+        if (cudaError_t e_ = launch_pdl(k_prefill_schedule_adjacent, dim3((a.n_items + 255) / 256), dim3(256), 0, s, a))
+            return e_;
+    }
     cudaError_t e = cudaGetLastError();
     if (e != cudaSuccess) return e;
     using L = Smem<kKStages, kVStages>;
@@ -606,7 +615,7 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s)
     e = cudaFuncSetAttribute(k_prefill_tc<kKStages, kVStages>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)smem);
     if (e != cudaSuccess) return e;
-    k_prefill_tc<kKStages, kVStages><<<(unsigned)a.n_items, kThreads, smem, s>>>(mq, mk, mv, a);
+    if (cudaError_t e_ = launch_pdl(k_prefill_tc<kKStages, kVStages>, dim3((unsigned)a.n_items), dim3(kThreads), smem, s, mq, mk, mv, a)) return e_;
     return cudaGetLastError();
 }
 

@@ -58,6 +58,8 @@ constexpr int BS = 64;   // block size (tokens); query and key blocks alike
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_block_stats(const RbsArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     constexpr int D = 128;
     __shared__ __align__(16) uint16_t tile[BS * D];
     __shared__ float cen[D];
@@ -113,6 +115,8 @@ __global__ void __launch_bounds__(256) k_block_stats(const RbsArgs a)
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_pool_q(const RbsArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     constexpr int D = 128;
     __shared__ float part[16][D];
     __shared__ float red[4];
@@ -165,6 +169,8 @@ constexpr int kPK = 32;    // K chunk
 template <bool QUANT>
 __global__ void __launch_bounds__(256) k_pair_tile(const RbsArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     constexpr int D = 128;
     __shared__ __align__(16) float sQ[kPK][kPT];
     __shared__ __align__(16) float sC[kPK][kPT];
@@ -302,6 +308,8 @@ __device__ __forceinline__ uint32_t *qstate_of(const RbsArgs &a, int arr)
 
 __global__ void __launch_bounds__(512) k_qhist(const RbsArgs a, int pass)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ unsigned hist[2048];
     const int arr = blockIdx.y;          // branch * Hq + h
     const size_t nP = (size_t)a.nB * (a.nB + 1) / 2;
@@ -331,6 +339,8 @@ __global__ void __launch_bounds__(512) k_qhist(const RbsArgs a, int pass)
 
 __global__ void __launch_bounds__(1024) k_qpick(const RbsArgs a, int pass)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ long long wt[33];
     __shared__ unsigned s_digit;
     __shared__ long long s_below;
@@ -388,6 +398,8 @@ __global__ void __launch_bounds__(1024) k_qpick(const RbsArgs a, int pass)
 // four 32-column words in flight per iteration
 __global__ void __launch_bounds__(256) k_mask_scores(const RbsArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= a.Hq * a.nB) return;
@@ -426,6 +438,8 @@ constexpr int kScanChunk = 1024;   // rows per CTA (one per thread)
 
 __global__ void __launch_bounds__(kScanChunk) k_csr_sum(const RbsArgs a, long long *chunk_sum)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ long long wt[33];
     const int R = a.Hq * a.nB;
     const int r = blockIdx.x * kScanChunk + threadIdx.x;
@@ -436,6 +450,8 @@ __global__ void __launch_bounds__(kScanChunk) k_csr_sum(const RbsArgs a, long lo
 
 __global__ void __launch_bounds__(1024) k_csr_chunks(const RbsArgs a, long long *chunk_sum, int nchunks)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ long long wt[33];
     long long run = 0;
     for (int c0 = 0; c0 < nchunks; c0 += 1024) {
@@ -455,6 +471,8 @@ __global__ void __launch_bounds__(1024) k_csr_chunks(const RbsArgs a, long long 
 
 __global__ void __launch_bounds__(kScanChunk) k_csr_scan(const RbsArgs a, const long long *chunk_off)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ long long wt[33];
     const int R = a.Hq * a.nB;
     const int r = blockIdx.x * kScanChunk + threadIdx.x;
@@ -465,6 +483,8 @@ __global__ void __launch_bounds__(kScanChunk) k_csr_scan(const RbsArgs a, const 
 
 __global__ void __launch_bounds__(256) k_csr_fill(const RbsArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= a.Hq * a.nB) return;
@@ -497,6 +517,8 @@ __global__ void __launch_bounds__(256) k_csr_fill(const RbsArgs a)
 
 __global__ void k_copy_tau(const RbsArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     const int h = threadIdx.x + blockIdx.x * blockDim.x;
     if (h >= a.Hq) return;
     a.tau[h] = a.tau_c[h];
@@ -505,6 +527,8 @@ __global__ void k_copy_tau(const RbsArgs a)
 
 __global__ void k_tau_out(const RbsArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     const int x = threadIdx.x + blockIdx.x * blockDim.x;
     if (x < 2 * a.Hq) a.tau_out[x] = a.tau[x];
 }
@@ -517,38 +541,40 @@ cudaError_t launch_rbs(const RbsArgs &a, cudaStream_t s)
     const bool quant = a.tau_c == nullptr;
     cudaError_t e;
     // per-kv-head block statistics on sequence 0's keys
-    k_block_stats<<<dim3(a.nB, a.c.Hkv), 256, 0, s>>>(a);
-    k_pool_q<<<dim3(a.nB, a.Hq), 256, 0, s>>>(a);
+    if (cudaError_t e_ = launch_pdl(k_block_stats, dim3(dim3(a.nB, a.c.Hkv)), dim3(256), 0, s, a)) return e_;
+    if (cudaError_t e_ = launch_pdl(k_pool_q, dim3(dim3(a.nB, a.Hq)), dim3(256), 0, s, a)) return e_;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int nTB = (a.nB + kPT - 1) / kPT;
     const int tiles = nTB * (nTB + 1) / 2;
     const size_t smem = 0;
     if (quant) {
-        k_pair_tile<true><<<dim3(tiles, a.Hq), 256, smem, s>>>(a);
+        if (cudaError_t e_ = launch_pdl(k_pair_tile<true>, dim3(dim3(tiles, a.Hq)), dim3(256), smem, s, a)) return e_;
         if ((e = cudaMemsetAsync(a.qhist, 0, (size_t)2 * a.Hq * (3 * 2048 + 4) * 4, s)) != cudaSuccess) return e;
         const size_t nP = (size_t)a.nB * (a.nB + 1) / 2;
         const dim3 hgrid((unsigned)((nP + kQChunk - 1) / kQChunk), 2 * a.Hq);
         for (int pass = 0; pass < 3; ++pass) {
-            k_qhist<<<hgrid, 512, 0, s>>>(a, pass);
-            k_qpick<<<2 * a.Hq, 1024, 0, s>>>(a, pass);
+            if (cudaError_t e_ = launch_pdl(k_qhist, dim3(hgrid), dim3(512), 0, s, a, pass)) return e_;
+            if (cudaError_t e_ = launch_pdl(k_qpick, dim3(2 * a.Hq), dim3(1024), 0, s, a, pass)) return e_;
         }
-        k_mask_scores<<<(a.Hq * a.nB + 7) / 8, 256, 0, s>>>(a);
+        if (cudaError_t e_ = launch_pdl(k_mask_scores, dim3((a.Hq * a.nB + 7) / 8), dim3(256), 0, s, a)) return e_;
     } else {
-        k_copy_tau<<<(a.Hq + 127) / 128, 128, 0, s>>>(a);
+        if (cudaError_t e_ = launch_pdl(k_copy_tau, dim3((a.Hq + 127) / 128), dim3(128), 0, s, a)) return e_;
         if ((e = cudaMemsetAsync(a.rowcnt, 0, (size_t)a.Hq * a.nB * sizeof(int32_t), s)) != cudaSuccess) return e;
-        k_pair_tile<false><<<dim3(tiles, a.Hq), 256, smem, s>>>(a);
+        if (cudaError_t e_ = launch_pdl(k_pair_tile<false>, dim3(dim3(tiles, a.Hq)), dim3(256), smem, s, a)) return e_;
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {
         const int R = a.Hq * a.nB;
         const int nch = (R + kScanChunk - 1) / kScanChunk;
         long long *chunk = reinterpret_cast<long long *>(a.rowcnt + R + 1 + ((R + 1) & 1));   // 8-byte aligned
-        k_csr_sum<<<nch, kScanChunk, 0, s>>>(a, chunk);
-        k_csr_chunks<<<1, 1024, 0, s>>>(a, chunk, nch);
-        k_csr_scan<<<nch, kScanChunk, 0, s>>>(a, chunk);
+        if (cudaError_t e_ = launch_pdl(k_csr_sum, dim3(nch), dim3(kScanChunk), 0, s, a, chunk)) return e_;
+        if (cudaError_t e_ = launch_pdl(k_csr_chunks, dim3(1), dim3(1024), 0, s, a, chunk, nch)) return e_;
+        if (cudaError_t e_ = launch_pdl(k_csr_scan, dim3(nch), dim3(kScanChunk), 0, s, a, chunk)) return e_;
     }
-    k_csr_fill<<<(a.Hq * a.nB + 7) / 8, 256, 0, s>>>(a);
-    if (a.tau_out) k_tau_out<<<(2 * a.Hq + 127) / 128, 128, 0, s>>>(a);
+    if (cudaError_t e_ = launch_pdl(k_csr_fill, dim3((a.Hq * a.nB + 7) / 8), dim3(256), 0, s, a)) return e_;
+    if (a.tau_out) {
+        if (cudaError_t e_ = launch_pdl(k_tau_out, dim3((2 * a.Hq + 127) / 128), dim3(128), 0, s, a)) return e_;
+    }
     return cudaGetLastError();
 }
 

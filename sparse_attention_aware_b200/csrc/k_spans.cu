@@ -19,6 +19,8 @@ constexpr int kMaxSpans = 1024;
 
 __global__ void __launch_bounds__(256) k_span_blocks(const SpanArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     __shared__ int2 rng[kMaxSpans];        // merged [start, end)
     __shared__ int ent_base[kMaxSpans + 1];
     __shared__ int tok_base[kMaxSpans + 1];
@@ -102,7 +104,7 @@ cudaError_t launch_spans(const SpanArgs &a, cudaStream_t s)
 {
     if (a.c.B == 0) return cudaSuccess;
     if (a.max_spans > kMaxSpans) return cudaErrorInvalidValue;
-    k_span_blocks<<<a.c.B, 256, 0, s>>>(a);
+    if (cudaError_t e_ = launch_pdl(k_span_blocks, dim3(a.c.B), dim3(256), 0, s, a)) return e_;
     return cudaGetLastError();
 }
 

@@ -76,6 +76,8 @@ constexpr uint64_t kScoreWaitNs = 1000ull * 1000 * 1000;   // 1 s
 template <int D, int HPG, bool QF32>
 __global__ void __launch_bounds__(ScoreGeom<D, HPG>::THREADS) k_topk_score(const TopkArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     using Gm = ScoreGeom<D, HPG>;
     constexpr int G = Gm::G, GPW = Gm::GPW, U = Gm::U, TT = Gm::TT, NS = Gm::NS, MAXJ = Gm::MAXJ;
     constexpr int HL = HPG == 1 ? 0 : HPG == 2 ? 1 : HPG == 4 ? 2 : 3;   // log2(HPG)
@@ -358,6 +360,8 @@ constexpr int kCandCap = 4096;
 // Dynamic shared memory: 2 bitmaps of Lcap bits + 2 x kCandCap words.
 __global__ void __launch_bounds__(kSelThreads, 2) k_topk_select(const TopkArgs a)
 {
+    pdl_wait();
+    pdl_trigger();
     extern __shared__ uint32_t dsm[];
     __shared__ unsigned hist[2048];
     __shared__ int warp_tot[33];
@@ -550,7 +554,7 @@ cudaError_t launch_score(const TopkArgs &a, cudaStream_t s)
     cudaError_t e = cudaFuncSetAttribute(k_topk_score<D, HPG, QF32>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    k_topk_score<D, HPG, QF32><<<grid, ScoreGeom<D, HPG>::THREADS, smem, s>>>(a);
+    if (cudaError_t e_ = launch_pdl(k_topk_score<D, HPG, QF32>, dim3(grid), dim3(ScoreGeom<D, HPG>::THREADS), smem, s, a)) return e_;
     return cudaGetLastError();
 }
 
@@ -582,7 +586,7 @@ cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s)
     const size_t smem = select_smem_bytes(Lcap);
     e = cudaFuncSetAttribute(k_topk_select, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
-    k_topk_select<<<a.c.B * a.Hq, kSelThreads, smem, s>>>(a);
+    if (cudaError_t e_ = launch_pdl(k_topk_select, dim3(a.c.B * a.Hq), dim3(kSelThreads), smem, s, a)) return e_;
     return cudaGetLastError();
 }
 

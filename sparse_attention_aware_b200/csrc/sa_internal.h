@@ -40,6 +40,10 @@ struct DecodeArgs {
     DevStatus *st;
 };
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+// block-list selections with at most 16 query heads per kv head: one CTA per
+// (split, kv head, sequence) on mma.sync (k_decode_gqa.cu)
+bool decode_gqa_supported(const DecodeArgs &a);
+cudaError_t launch_decode_gqa_split(const DecodeArgs &a, cudaStream_t s);
 
 // ---- top-k ------------------------------------------------------------------
 struct TopkArgs {

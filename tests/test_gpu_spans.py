@@ -132,3 +132,58 @@ def test_masked_decode_full_size_steps(cuda_dev):
         ref, _ = oracle.decode_members(cv, q, want, scale, rows=rows)
         assert_close_attn(out.float().cpu().numpy().reshape(-1, d)[rows], ref)
     ws.raise_on_fault()
+
+
+@pytest.mark.parametrize("d,Hq,Hkv,qdt", [
+    (128, 8, 8, torch.bfloat16),     # one query head per kv head
+    (128, 8, 4, torch.bfloat16),
+    (128, 16, 4, torch.bfloat16),
+    (64, 32, 2, torch.bfloat16),     # 16 query heads per kv head (all MMA rows used)
+    (128, 8, 1, torch.float32),      # fp32 query (high + low bf16 parts)
+    (128, 32, 1, torch.bfloat16),    # 32 per kv head: per-head kernel
+])
+def test_masked_decode_group_shapes(cuda_dev, d, Hq, Hkv, qdt):
+    lens = [700, 4100, 33, 2500]
+    P = 16
+    cache, q = W.random_decode(90 + Hq + d, len(lens), Hq, Hkv, d, lens, P, q_dtype=qdt)
+    Lmax = cache.max_pages * P
+    gc = cache.to(cuda_dev)
+    ws = sa.Workspace(cuda_dev)
+    scale = 1 / math.sqrt(d)
+    prod = [SP.spans_for(SP.GLOBAL, lens[0], 2048), SP.spans_for(SP.FOCUS, lens[1], 2048, 3, [0, 1]),
+            SP.spans_for(SP.STREAMING, lens[2], 2048), SP.spans_for(SP.LOCAL, lens[3], 2048)]
+    spans, cnt, rnd = SP.pack(prod, cuda_dev)
+    sel = sa.select_blocks_spans(gc, spans, cnt, rnd, ws=ws)
+    mem = _members_from_blocks(sel.blocks.cpu().numpy(), sel.block_counts.cpu().numpy(), P, Lmax)
+    ref, ref_lse = oracle.decode_members(cache, q, mem, scale)
+    for S in (1, 3, 8):
+        out, lse = sa.sparse_decode_attn(gc, q.to(cuda_dev), sel, scale, S, ws=ws)
+        assert_close_attn(out.float().cpu().numpy().reshape(-1, d), ref)
+        np.testing.assert_allclose(lse.cpu().numpy().reshape(-1), ref_lse, atol=2e-3, rtol=0)
+    ws.raise_on_fault()
+
+
+def test_masked_decode_empty_and_malformed_lists(cuda_dev):
+    """An empty list gives a zero output and lse = -inf; a malformed entry is
+    recorded as a device fault and skipped, the rest still attends."""
+    lens = [500, 900]
+    P, d = 16, 128
+    cache, q = W.random_decode(5, 2, 8, 1, d, lens, P)
+    gc = cache.to(cuda_dev)
+    blocks = torch.zeros((2, 4, 4), dtype=torch.int32)
+    blocks[1, 0] = torch.tensor([0, 0, 16, 0])
+    blocks[1, 1] = torch.tensor([3, 9, 4, 16])       # lo > hi: malformed
+    blocks[1, 2] = torch.tensor([5, 2, 10, 16])
+    counts = torch.tensor([0, 3], dtype=torch.int32)
+    sel = sa.BlockSelection(blocks.to(cuda_dev), counts.to(cuda_dev))
+    ws = sa.Workspace(cuda_dev)
+    out, lse = sa.sparse_decode_attn(gc, q.to(cuda_dev), sel, 0.1, 2, ws=ws)
+    st, det = ws.status()
+    assert st == 5 and det[1] == 5            # SA_ERR_DEVICE_FAULT, malformed block entry
+    o = out.float().cpu()
+    assert torch.all(o[0] == 0) and torch.all(torch.isinf(lse.cpu()[0]))
+    mem = np.zeros((2, cache.max_pages * P), dtype=np.uint8)
+    mem[1, 0:16] = 1
+    mem[1, 5 * 16 + 2:5 * 16 + 10] = 1
+    ref, _ = oracle.decode_members(cache, q, mem, 0.1)
+    assert_close_attn(o.numpy().reshape(-1, d)[8:], ref.reshape(-1, d)[8:])
