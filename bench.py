@@ -452,6 +452,8 @@ def main():
     if traffic:
         result["roofline"]["traffic"] = traffic.get("k_prefill_tc")
         result["roofline_decode"]["traffic"] = traffic.get("decode")
+    result["roofline"]["traffic_unit"] = "DRAM bytes per launch (ncu, full-size workload)"
+    result["roofline_decode"]["traffic_unit"] = "DRAM bytes per decode group (ncu, full-size workload)"
 
     if not args.no_e2e:
         result["e2e"] = e2e(step, dec, pre, msk, cfg, args, world, dev, dist if world > 1 else None)
@@ -464,15 +466,38 @@ def main():
         dist.destroy_process_group()
 
 
+# kernel sources each traffic figure was measured on; a figure is reported only
+# while these files are unchanged (see profiles/traffic.json)
+TRAFFIC_SOURCES = {
+    "k_prefill_tc": ["k_prefill_tc.cu", "tc_ptx.cuh", "sa_common.cuh"],
+    "decode": ["k_topk.cu", "k_decode.cu", "sa_common.cuh", "tc_ptx.cuh"],
+}
+
+
+def sources_sha1(files):
+    import hashlib
+    h = hashlib.sha1()
+    for f in files:
+        with open(os.path.join(ROOT, "sparse_attention_aware_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
+
+
 def load_traffic():
-    """Per-launch DRAM bytes (read + write) from the committed ncu summary, if
-    it matches the current kernels; None otherwise."""
+    """Per-launch DRAM bytes (read + write) from the committed ncu summary,
+    for each kernel whose sources still hash to the recorded value; None where
+    the kernel has changed since the counters were taken."""
     p = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(p):
         return None
     try:
         with open(p) as f:
-            return json.load(f)
+            rec = json.load(f)
+        out = {}
+        for key, files in TRAFFIC_SOURCES.items():
+            r = rec.get(key)
+            out[key] = r["bytes"] if r and r.get("src_sha1") == sources_sha1(files) else None
+        return out
     except Exception:
         return None
 

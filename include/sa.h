@@ -37,6 +37,13 @@
  *  - Determinism: results are bitwise reproducible run to run (fixed split
  *    and reduction orders, no floating-point atomics).
  *  - Device: the current CUDA device; all pointers must live on it.
+ *  - Launch: every kernel is launched with programmatic dependent launch
+ *    allowed ([LoZA] "四、从外卖到AI" names PDL) and waits for the previous
+ *    kernel in the stream to complete before it touches memory; it lets the
+ *    next kernel be scheduled early.  A caller's kernel launched after it
+ *    with the programmatic attribute must itself wait (griddepcontrol.wait /
+ *    cudaGridDependencySynchronize) before reading these outputs; kernels
+ *    launched without the attribute are ordered as usual.
  */
 #ifndef SA_H_
 #define SA_H_
@@ -224,6 +231,11 @@ SA_API sa_status sa_select_blocks(const sa_kv_cache *kv, const sa_block_select_a
  * The set is cut into num_splits contiguous parts (split-KV); every part
  * yields (max, sum, partial output) and a combine pass merges them.  An
  * empty set gives out = 0 and lse = -inf.
+ * Block lists (one list per sequence, shared by every head) with at most 16
+ * query heads per kv head are computed per GQA group on tensor cores: the
+ * parts are runs of list entries balanced by entry count, S = q.k is
+ * accumulated in fp32 (an fp32 query as bf16 high + low parts), and the
+ * softmax weights enter the P.V product as bf16.
  *   q        [batch][num_q_heads][head_dim], fp32 or bf16
  *   out      bf16 [batch][num_q_heads][head_dim]
  *   lse_out  fp32 [batch][num_q_heads] natural log, nullable
