@@ -383,6 +383,7 @@ def main():
     qe.record(stream)
     torch.cuda.synchronize()
     rbs_quant_ms = qs.elapsed_time(qe) / 5
+    da_us = da_state_cost(cfg, dev)
     total_ms = t_start.elapsed_time(t_end)
     parts = {"decode": 0.0, "masked": 0.0, "rbs_select": 0.0, "prefill": 0.0}
     for e in evs:
@@ -435,7 +436,8 @@ def main():
                        "frac_hbm": round(K * rbs_bytes / (rbs_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
         "masked_decode": {"ms_per_step": round(msk_ms / K, 4),
                           "gbs": round(world * msk_bytes / (msk_ms * 1e-3) / 1e9, 2),
-                          "frac_hbm": round(msk_bytes / (msk_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4)},
+                          "frac_hbm": round(msk_bytes / (msk_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                          "da_state_host_us_per_step": round(da_us, 2)},
         "roofline": {"bound": "tensor", "kernel": "k_prefill_tc", "achieved": round(per_gpu_pre, 2),
                      "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                      "frac": round(per_gpu_pre / pk["bf16_tflops_sustained"], 4), "traffic": None,
@@ -464,6 +466,26 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def da_state_cost(cfg, dev, steps=256):
+    """Host time per decode step of the DA state machine for the masked-decode
+    batch (observe one token per sequence, build the next step's spans, pack
+    them into device tensors), over a scripted stream that cycles through
+    focus, local and global declarations."""
+    import time
+    from sparse_attention_aware_b200 import da_state as DA
+    m = cfg.msk
+    V = DA.DAVocab()
+    script = [V.focus_open, V.chunk_base + 3, V.chunk_base + 17, V.focus_close, 11, 12, V.local_tag, 13, 14,
+              V.global_tag, 15, 16]
+    batch = DA.DABatch([m["L"] - steps] * m["B"])
+    lens = [m["L"] - steps] * m["B"]
+    t0 = time.perf_counter()
+    for i in range(steps):
+        lens = [L + 1 for L in lens]
+        batch.step([script[(i + b) % len(script)] for b in range(m["B"])], lens, device=dev, max_spans=2)
+    return (time.perf_counter() - t0) / steps * 1e6
 
 
 # kernel sources each traffic figure was measured on; a figure is reported only

@@ -46,13 +46,17 @@ def spans_for(mode: str, seq_len: int, chunk: int = 2048, origin: int = 0,
 def pack(span_lists: Sequence[Sequence[Tuple[int, int, bool]]], device="cuda", max_spans: int = 0):
     """Pack per-sequence span lists into (spans int32 [B][S][2], counts int32 [B],
     round uint8 [B][S]) tensors for ``select_blocks_spans``."""
+    import numpy as np
     B = len(span_lists)
     S = max([max_spans] + [len(s) for s in span_lists] + [1])
-    spans = torch.zeros((B, S, 2), dtype=torch.int32)
-    rnd = torch.zeros((B, S), dtype=torch.uint8)
-    cnt = torch.zeros((B,), dtype=torch.int32)
+    spans = np.zeros((B, S, 2), dtype=np.int32)
+    rnd = np.zeros((B, S), dtype=np.uint8)
+    cnt = np.zeros((B,), dtype=np.int32)
     for b, lst in enumerate(span_lists):
-        cnt[b] = len(lst)
-        for i, (s0, s1, r) in enumerate(lst):
-            spans[b, i, 0], spans[b, i, 1], rnd[b, i] = s0, s1, int(bool(r))
-    return spans.to(device), cnt.to(device), rnd.to(device)
+        n = len(lst)
+        cnt[b] = n
+        if n:
+            spans[b, :n] = [(s0, s1) for s0, s1, _ in lst]
+            rnd[b, :n] = [1 if r else 0 for _, _, r in lst]
+    return (torch.from_numpy(spans).to(device), torch.from_numpy(cnt).to(device),
+            torch.from_numpy(rnd).to(device))

@@ -187,3 +187,51 @@ def test_masked_decode_empty_and_malformed_lists(cuda_dev):
     mem[1, 5 * 16 + 2:5 * 16 + 10] = 1
     ref, _ = oracle.decode_members(cache, q, mem, 0.1)
     assert_close_attn(o.numpy().reshape(-1, d)[8:], ref.reshape(-1, d)[8:])
+
+
+def test_da_state_machine_drives_masked_decode(cuda_dev):
+    """Scripted tag streams -> host DA state machine -> GPU block lists and
+    decode, step by step over growing sequences; the oracle side takes the
+    modes written out by hand and builds its spans with oracle.modes."""
+    from sparse_attention_aware_b200 import da_state as DA
+    V = DA.DAVocab()
+    G, LOC, FO, FC = V.global_tag, V.local_tag, V.focus_open, V.focus_close
+    C = lambda c: V.chunk_base + c
+    prompts = [6000, 9000, 4500]
+    streams = [[FO, C(0), C(2), FC, 5, LOC],
+               [LOC, 1, G, FO, C(3), FC],
+               [7, FO, C(1), FC, G, 2]]
+    # mode in effect for each step's read, per the stream above
+    modes = [[(OM.GLOBAL, ()), (OM.GLOBAL, ()), (OM.GLOBAL, ()), (OM.FOCUS, (0, 2)), (OM.FOCUS, (0, 2)),
+              (OM.LOCAL, ())],
+             [(OM.LOCAL, ()), (OM.LOCAL, ()), (OM.GLOBAL, ()), (OM.GLOBAL, ()), (OM.GLOBAL, ()),
+              (OM.FOCUS, (3,))],
+             [(OM.GLOBAL, ()), (OM.GLOBAL, ()), (OM.GLOBAL, ()), (OM.FOCUS, (1,)), (OM.GLOBAL, ()),
+              (OM.GLOBAL, ())]]
+    steps = 6
+    Hq, Hkv, d, P = 16, 2, 128, 16
+    cap = [L + steps for L in prompts]
+    cache, _ = W.random_decode(123, len(prompts), Hq, Hkv, d, cap, P)
+    Lmax = cache.max_pages * P
+    g = torch.Generator().manual_seed(321)
+    machine = DA.DABatch(prompts)
+    ws = sa.Workspace(cuda_dev)
+    scale = 1 / math.sqrt(d)
+    for i in range(steps):
+        lens = [L + i + 1 for L in prompts]
+        step_cache = W.PagedCache(cache.k, cache.v, cache.page_table, torch.tensor(lens, dtype=torch.int32))
+        gc = step_cache.to(cuda_dev)
+        spans, cnt, rnd = machine.step([s[i] for s in streams], lens, device=cuda_dev)
+        sel = sa.select_blocks_spans(gc, spans, cnt, rnd, ws=ws)
+        want = np.zeros((len(prompts), Lmax), dtype=np.uint8)
+        for b, L in enumerate(lens):
+            m, ch = modes[b][i]
+            want[b, :L] = oracle.span_members(L, P, OM.mode_spans(m, L, 2048, 0, ch))
+        got = _members_from_blocks(sel.blocks.cpu().numpy(), sel.block_counts.cpu().numpy(), P, Lmax)
+        np.testing.assert_array_equal(got, want)
+        q = torch.randn((len(prompts), Hq, d), generator=g).to(torch.bfloat16)
+        out, lse = sa.sparse_decode_attn(gc, q.to(cuda_dev), sel, scale, 4, ws=ws)
+        ref, ref_lse = oracle.decode_members(step_cache, q, want, scale)
+        assert_close_attn(out.float().cpu().numpy().reshape(-1, d), ref)
+        np.testing.assert_allclose(lse.cpu().numpy().reshape(-1), ref_lse, atol=2e-3, rtol=0)
+    ws.raise_on_fault()
