@@ -384,6 +384,7 @@ def main():
     torch.cuda.synchronize()
     rbs_quant_ms = qs.elapsed_time(qe) / 5
     da_us = da_state_cost(cfg, dev)
+    tiered = tiered_measure(msk, cfg, dev)
     total_ms = t_start.elapsed_time(t_end)
     parts = {"decode": 0.0, "masked": 0.0, "rbs_select": 0.0, "prefill": 0.0}
     for e in evs:
@@ -438,6 +439,7 @@ def main():
                           "gbs": round(world * msk_bytes / (msk_ms * 1e-3) / 1e9, 2),
                           "frac_hbm": round(msk_bytes / (msk_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                           "da_state_host_us_per_step": round(da_us, 2)},
+        "tiered_kv": tiered,
         "roofline": {"bound": "tensor", "kernel": "k_prefill_tc", "achieved": round(per_gpu_pre, 2),
                      "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
                      "frac": round(per_gpu_pre / pk["bf16_tflops_sustained"], 4), "traffic": None,
@@ -466,6 +468,75 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def tiered_measure(msk, cfg, dev, steps=64, slot_frac=0.125):
+    """Tiered KV on the masked-decode cache: the whole cache in a pinned host
+    tier, ``slot_frac`` of its pages as device slots.  A scripted DA stream
+    per sequence (focus on two chunks for 8 steps, then local for 8 steps, the
+    chunks moving on each cycle; the first token is <local>, so no step reads
+    globally) drives span selection and decode; missing
+    pages are fetched on the tier's copy stream before each step.  Reports the
+    hit rate, fetched bytes, the fetch kernel's host-link rate and the time
+    per step of the whole loop (fetch + select + decode)."""
+    import torch
+    import sparse_attention_aware_b200 as sa
+    from sparse_attention_aware_b200 import da_state as DA, spans as SP, tiered as T
+    m = cfg.msk
+    P, L = m["P"], m["L"]
+    n_pages = int(msk.cache.page_table.numel())
+    tier = T.TieredKV(msk.cache, slots=max(1, int(slot_frac * n_pages)), device=dev, time_fetches=True)
+    V = DA.DAVocab()
+    n_chunks = L // 2048
+    machines = [DA.DAStateMachine(L - steps) for _ in range(m["B"])]
+    ws = sa.Workspace(dev)
+    out = torch.empty((m["B"], m["Hq"], m["d"]), dtype=torch.bfloat16, device=dev)
+
+    def tokens(i, b):
+        # per 16 steps: <local>, a focus declaration on chunks (c0, c0 + 1)
+        # read for 8 steps, then <local> again; never global
+        cyc, ph = divmod(i, 16)
+        c0 = (7 * b + 5 * cyc) % (n_chunks - 1)
+        script = [V.local_tag, V.focus_open, V.chunk_base + c0, V.chunk_base + c0 + 1, V.focus_close]
+        if ph < len(script):
+            return script[ph]
+        return V.local_tag if ph == 12 else 100 + ph
+
+    def one(i, timed):
+        lens = [L - steps + i + 1] * m["B"]
+        lists = []
+        for b, mach in enumerate(machines):
+            mach.observe(tokens(i, b))
+            lists.append(mach.next_spans(lens[b]))
+        spans, cnt, rnd = SP.pack(lists, dev, max_spans=2)
+        tier.prepare([T.span_pages(l, n, P) for l, n in zip(lists, lens)])
+        c = tier.cache
+        sel = sa.select_blocks_spans(c, spans, cnt, rnd, ws=ws)
+        sa.sparse_decode_attn(c, msk.q_steps[i % msk.q_steps.shape[0]], sel, 1 / math.sqrt(m["d"]), 8,
+                              out=out, want_lse=False, ws=ws)
+
+    for i in range(4):           # warm-up: first fetches, no timing
+        one(i, False)
+    torch.cuda.synchronize()
+    tier.map.stats = {"hits": 0, "misses": 0}
+    fb0 = tier.fetched_bytes
+    tier.fetch_events = []
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record()
+    for i in range(4, steps):
+        one(i, True)
+    t1.record()
+    torch.cuda.synchronize()
+    ws.raise_on_fault("tiered masked decode")
+    fetch_ms = sum(a.elapsed_time(b) for a, b in tier.fetch_events)
+    st = tier.map.stats
+    fetched = tier.fetched_bytes - fb0
+    return {"slots": tier.map.slots, "pages": n_pages, "device_kv_fraction": round(tier.map.slots / n_pages, 4),
+            "steps": steps - 4, "hit_rate": round(st["hits"] / max(1, st["hits"] + st["misses"]), 4),
+            "fetched_mb_per_step": round(fetched / (steps - 4) / 1e6, 3),
+            "fetch_gbs": round(fetched / max(fetch_ms, 1e-9) / 1e6, 2),
+            "ms_per_step": round(t0.elapsed_time(t1) / (steps - 4), 4),
+            "note": "whole loop incl. host DA state machine, span packing, page-table publish and fetch"}
 
 
 def da_state_cost(cfg, dev, steps=256):

@@ -312,6 +312,33 @@ SA_API sa_status sa_sparse_prefill_attn(const sa_kv_cache *kv, const void *q, in
                                  sa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* 5. sa_fetch_pages -- bring KV pages from a host tier into device slots   */
+/* ------------------------------------------------------------------------ */
+/*
+ * [DA-1] (a step only hides context, it deletes none, so the KV pages no
+ * step is reading can sit in an outer memory tier and be fetched back,
+ * overlapped with decoding, when a declaration names them again); [DA-2]
+ * "对百万上下文产品意味着什么" (the KV cache as tiered storage: recent content
+ * in HBM, focus regions loaded on demand, far history in CPU memory).
+ * For pair i = {src, dst} (int32 [n][2] in device memory), page src of the
+ * host tier goes to page slot dst of the device pools, K and V alike:
+ *   host_k, host_v  page-major arrays of page_bytes-sized pages in pinned host
+ *                   memory the device reads at the same address (cudaHostAlloc
+ *                   / cudaMallocHost / a pinned torch tensor, with unified
+ *                   addressing); host_pages pages each
+ *   dev_k, dev_v    the cache pools (kv->k, kv->v layout), dev_pages slots
+ *   page_bytes      num_kv_heads*page_size*head_dim*2, a multiple of 16
+ * One kernel gathers every pair with 16-byte loads over the host link (no
+ * per-page copy calls).  A pair whose src is outside [0, host_pages) or whose
+ * dst is outside [0, dev_pages) is skipped and recorded as
+ * SA_ERR_DEVICE_FAULT in ws.  Two pairs must not name the same dst.
+ *   ws  any workspace of at least 256 bytes (only its status word is used).
+ */
+SA_API sa_status sa_fetch_pages(const void *host_k, const void *host_v, void *dev_k, void *dev_v,
+                                const int32_t *pairs, int32_t n, int64_t host_pages, int64_t dev_pages,
+                                size_t page_bytes, void *ws, size_t ws_bytes, sa_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Workspace sizing, status                                                 */
 /* ------------------------------------------------------------------------ */
 typedef enum {

@@ -193,6 +193,28 @@ def sparse_decode_attn(cache, q: torch.Tensor, sel, scale: Optional[float] = Non
     return out, lse
 
 
+def fetch_pages(host_k: torch.Tensor, host_v: torch.Tensor, dev_k: torch.Tensor, dev_v: torch.Tensor,
+                pairs: torch.Tensor, ws: Optional[Workspace] = None, stream=None) -> None:
+    """Copy host-tier pages into device page slots (``sa_fetch_pages``).
+    host_k/host_v: pinned CPU tensors [host_pages][Hkv][P][d] bf16; dev_k/dev_v:
+    device pools [slots][Hkv][P][d]; pairs: device int32 [n][2] {host page, slot}."""
+    if not (host_k.is_pinned() and host_v.is_pinned()):
+        raise ValueError("the host tier must be pinned memory")
+    if host_k.shape[1:] != dev_k.shape[1:] or host_v.shape != host_k.shape or dev_v.shape != dev_k.shape:
+        raise ValueError("host tier and device pool pages differ in shape")
+    if host_k.dtype != torch.bfloat16 or dev_k.dtype != torch.bfloat16 or host_v.dtype != torch.bfloat16 \
+            or dev_v.dtype != torch.bfloat16:
+        raise ValueError("KV pages are bf16")
+    if pairs.dtype != torch.int32 or pairs.dim() != 2 or pairs.shape[1] != 2 or not pairs.is_contiguous():
+        raise ValueError("pairs must be a contiguous int32 [n][2] tensor")
+    page_bytes = host_k[0].numel() * 2 if host_k.shape[0] else dev_k[0].numel() * 2
+    w = _ws(ws, dev_k.device)
+    wp, wn = w.aligned(256)
+    _check(L.load().sa_fetch_pages(host_k.data_ptr(), host_v.data_ptr(), dev_k.data_ptr(), dev_v.data_ptr(),
+                                   pairs.data_ptr(), pairs.shape[0], host_k.shape[0], dev_k.shape[0], page_bytes,
+                                   wp, wn, _stream(stream)), "sa_fetch_pages")
+
+
 def select_blocks_spans(cache, spans: torch.Tensor, span_counts: torch.Tensor, span_round: torch.Tensor,
                         max_blocks: Optional[int] = None, out: Optional[BlockSelection] = None,
                         ws: Optional[Workspace] = None, stream=None) -> BlockSelection:

@@ -146,6 +146,31 @@ size_t sa_workspace_bytes(sa_op op, const sa_kv_cache *kv, const sa_ws_query *q)
     }
 }
 
+sa_status sa_fetch_pages(const void *host_k, const void *host_v, void *dev_k, void *dev_v, const int32_t *pairs,
+                         int32_t n, int64_t host_pages, int64_t dev_pages, size_t page_bytes, void *ws,
+                         size_t ws_bytes, sa_stream_t stream)
+{
+    if (n < 0 || host_pages < 0 || dev_pages < 0 || page_bytes == 0 || page_bytes % 16) return SA_ERR_INVALID_ARGUMENT;
+    if (n > 0 && (!host_k || !host_v || !dev_k || !dev_v || !pairs)) return SA_ERR_INVALID_ARGUMENT;
+    if (!aligned(host_k, 16) || !aligned(host_v, 16) || !aligned(dev_k, 16) || !aligned(dev_v, 16) ||
+        !aligned(pairs, 8))
+        return SA_ERR_INVALID_ARGUMENT;
+    sa_status st = check_ws(ws, ws_bytes, kHeader);
+    if (st != SA_OK) return st;
+    FetchArgs a{};
+    a.host_k = host_k;
+    a.host_v = host_v;
+    a.dev_k = dev_k;
+    a.dev_v = dev_v;
+    a.pairs = pairs;
+    a.n = n;
+    a.host_pages = host_pages;
+    a.dev_pages = dev_pages;
+    a.page_bytes = page_bytes;
+    a.st = static_cast<DevStatus *>(ws);
+    return cuda_status(launch_fetch(a, (cudaStream_t)stream));
+}
+
 sa_status sa_workspace_init(void *ws, size_t ws_bytes, sa_stream_t stream)
 {
     if (!ws || ws_bytes < kHeader || !aligned(ws, kAlign)) return SA_ERR_WORKSPACE;

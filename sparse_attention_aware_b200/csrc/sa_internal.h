@@ -40,6 +40,18 @@ struct DecodeArgs {
     DevStatus *st;
 };
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+
+// ---- host-tier page fetch ---------------------------------------------------
+struct FetchArgs {
+    const void *host_k, *host_v;   // pinned host memory, device-readable
+    void *dev_k, *dev_v;
+    const int32_t *pairs;          // [n][2] {host page, device slot}
+    int n;
+    long long host_pages, dev_pages;
+    size_t page_bytes;
+    DevStatus *st;
+};
+cudaError_t launch_fetch(const FetchArgs &a, cudaStream_t s);
 // block-list selections with at most 16 query heads per kv head: one CTA per
 // (split, kv head, sequence) on mma.sync (k_decode_gqa.cu)
 bool decode_gqa_supported(const DecodeArgs &a);
