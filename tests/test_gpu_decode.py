@@ -204,3 +204,30 @@ def test_gqa_decode_full_size(cuda_dev):
         assert_close_attn(out.float().cpu().numpy().reshape(-1, 128), ref)
         np.testing.assert_allclose(lse.cpu().numpy().reshape(-1), ref_lse, atol=2e-3, rtol=0)
     ws.raise_on_fault()
+
+
+# --------------------------------------------------------------------------
+# The bench's decode configuration, in the bench's launch configuration:
+# B=32, 32/8 heads, d=128, L=65536, 16-token shuffled pages, top-k 4096 per
+# query head, 8 splits.  Top-k bit-exact on every row; the anchor layer and a
+# reuse layer checked on sampled rows.
+# --------------------------------------------------------------------------
+def test_bench_decode_config(cuda_dev):
+    wl = W.gqa_decode(1005, device=cuda_dev, B=32, Hq=32, Hkv=8, d=128, L=65536, P=16, k=4096, layers=2,
+                      num_splits=8)
+    cpu = wl.cache.to("cpu")
+    q0, _ = enforce_gap(cpu, wl.q_layers[0].cpu(), wl.k, 1005)
+    ref_idx, ref_cnt = oracle.select_topk(cpu, q0, wl.k)
+    ws = sa.Workspace(cuda_dev)
+    sel = sa.select_topk(wl.cache, q0.to(cuda_dev), wl.k, ws=ws)
+    np.testing.assert_array_equal(sel.count.cpu().numpy(), ref_cnt)
+    np.testing.assert_array_equal(sel.idx.cpu().numpy(), ref_idx)
+    rows = np.random.default_rng(11).choice(32 * 32, 64, replace=False)
+    scale = 1 / math.sqrt(128)
+    for li, q in enumerate([q0, wl.q_layers[1].cpu()]):
+        v = wl.v_layers[li]
+        ref, ref_lse = oracle.decode_tokens(cpu, q, ref_idx, ref_cnt, scale, v=v.cpu(), rows=rows)
+        out, lse = sa.sparse_decode_attn(wl.cache.with_v(v), q.to(cuda_dev), sel, scale, wl.num_splits, ws=ws)
+        assert_close_attn(out.float().cpu().numpy().reshape(-1, 128)[rows], ref)
+        np.testing.assert_allclose(lse.cpu().numpy().reshape(-1)[rows], ref_lse, atol=2e-3, rtol=0)
+    ws.raise_on_fault()

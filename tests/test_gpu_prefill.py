@@ -126,3 +126,42 @@ def test_prefill_block_sparse_full_size_sampled(cuda_dev):
     hs = rng.integers(0, Hq, len(ts))
     rows = (ts * Hq + hs).astype(np.int64)
     _run(cuda_dev, wl, mask, rows=rows)
+
+
+def test_bench_prefill_config(cuda_dev):
+    """The bench's prefill configuration: 131072 tokens, 32/4 heads, 64x64
+    blocks, clustered keys with outliers, thresholds started at the bench's
+    quantile levels 0.965 / 0.985 and moved into >= 1e-3 gaps of the fp64
+    scores (the fp32 pair-score error is ~1e-4; near the 96.5% quantile of
+    2.1M pairs the scores lie ~1e-5 apart, so the nearest such gap sits in
+    the tail and the kept density comes out near 2% rather than the bench's
+    5%).  The RBS mask is compared bit for bit, the prefill output on
+    sampled rows."""
+    wl = W.clustered_prefill(1005, device=cuda_dev, T=131072, Hq=32, Hkv=4, d=128, block=64)
+    T, Hq, d = wl.q.shape
+    scale = 1 / math.sqrt(128)
+    cpu = wl.cache.to("cpu")
+    qc = wl.q.cpu()
+    c, r = oracle.block_stats(cpu, 64)
+    qbar, qn = oracle.pool_q(qc, 64)
+    Sc, Sr = oracle.pair_scores(qbar, qn, c, r, scale)
+    tc = [tau_in_gap(Sc[h], 0.965)[0] for h in range(Hq)]
+    tr = [tau_in_gap(Sr[h], 0.985)[0] for h in range(Hq)]
+    mask = oracle.rbs_mask(Sc, Sr, tc, tr, True, True)
+    assert 0.01 < mask.mean() < 0.08
+    ws = sa.Workspace(cuda_dev)
+    csr = sa.select_blocks_rbs(wl.cache, wl.q, 64, scale, tau_c=torch.tensor(tc), tau_r=torch.tensor(tr), ws=ws)
+    ws.raise_on_fault()
+    nB = T // 64
+    got = csr_to_mask(csr.row_ptr.cpu().numpy(), csr.cols.cpu().numpy(), Hq, nB)
+    np.testing.assert_array_equal(got, mask)
+    out, lse = sa.sparse_prefill_attn(wl.cache, wl.q, csr, scale, ws=ws)
+    ws.raise_on_fault()
+    rng = np.random.default_rng(13)
+    ts = np.concatenate([[0, 63, 64, T - 1, T - 64], rng.integers(0, T, 200)])
+    hs = rng.integers(0, Hq, len(ts))
+    rows = (ts * Hq + hs).astype(np.int64)
+    ref, ref_lse = oracle.prefill(cpu, qc, 64, mask, scale, rows=rows)
+    g_out = out.float().cpu().numpy().reshape(-1, d)[rows]
+    assert_close_attn(g_out, ref)
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(-1)[rows], ref_lse, atol=2e-3, rtol=0)
