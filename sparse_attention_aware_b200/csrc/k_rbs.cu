@@ -166,54 +166,87 @@ __device__ __forceinline__ void tri_index(int x, int &I, int &J)
 constexpr int kPT = 128;   // tile edge (blocks)
 constexpr int kPK = 32;    // K chunk
 
+constexpr int kPS = kPK + 2;   // shared row stride (floats): 8-byte column reads hit 32 distinct banks
+constexpr int kPairSmem = 2 * 2 * kPT * kPS * 4;   // 2 stages x (qbar, c) chunks
+
+__device__ __forceinline__ void cp_async8(uint32_t dst, const void *src, bool pred)
+{
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(pred ? 8 : 0)
+                 : "memory");
+}
+
+// Pooled dot products of one 128x128 tile of (query block, key block) pairs:
+// 32-wide chunks of d stream into a double-buffered shared-memory tile with
+// cp.async (rows padded to kPS floats), each thread accumulating 8 query
+// rows x 8 key columns (columns tx + 16*cc, so a warp's 8-byte column reads
+// cover all banks once) in ascending d order.
 template <bool QUANT>
-__global__ void __launch_bounds__(256) k_pair_tile(const RbsArgs a)
+__global__ void __launch_bounds__(256, 2) k_pair_tile(const RbsArgs a)
 {
     pdl_wait();
     pdl_trigger();
     constexpr int D = 128;
-    __shared__ __align__(16) float sQ[kPK][kPT];
-    __shared__ __align__(16) float sC[kPK][kPT];
+    extern __shared__ __align__(16) float psm[];
     int I, J;
     tri_index(blockIdx.x, I, J);
     const int h = blockIdx.y;
     const int g = h / (a.Hq / a.c.Hkv);
-    const int tid = threadIdx.x;
+    const int tid = threadIdx.x, lane = tid & 31;
     const int ty = tid >> 4, tx = tid & 15;
+    const float *qb = a.qbar + (size_t)h * a.nB * D;
+    const float *cb = a.cen + (size_t)g * a.nB * D;
+    const uint32_t sb = (uint32_t)__cvta_generic_to_shared(psm);
+
+    // chunk k0 of both operands into stage st: 128 rows x 16 pieces of 8 bytes each
+    auto load = [&](int k0, int st) {
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const int x = tid + 256 * u;
+            const int r = x >> 4, pc = x & 15;
+            const int i = I * kPT + r, j = J * kPT + r;
+            const uint32_t off = (uint32_t)((st * 2 * kPT + r) * kPS + pc * 2) * 4;
+            cp_async8(sb + off, qb + (size_t)(i < a.nB ? i : 0) * D + k0 + pc * 2, i < a.nB);
+            cp_async8(sb + off + kPT * kPS * 4, cb + (size_t)(j < a.nB ? j : 0) * D + k0 + pc * 2, j < a.nB);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+
     float acc[8][8];
 #pragma unroll
     for (int r = 0; r < 8; ++r)
 #pragma unroll
         for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
-    const float *qb = a.qbar + (size_t)h * a.nB * D;
-    const float *cb = a.cen + (size_t)g * a.nB * D;
+
+    load(0, 0);
 #pragma unroll 1
-    for (int k0 = 0; k0 < D; k0 += kPK) {
-        for (int x = tid; x < kPT * (kPK / 4); x += 256) {
-            const int r = x & (kPT - 1), kq = x >> 7;   // row in tile, float4 index in chunk
-            const int i = I * kPT + r, j = J * kPT + r;
-            float4 qv = make_float4(0, 0, 0, 0), cv = make_float4(0, 0, 0, 0);
-            if (i < a.nB) qv = *reinterpret_cast<const float4 *>(qb + (size_t)i * D + k0 + kq * 4);
-            if (j < a.nB) cv = *reinterpret_cast<const float4 *>(cb + (size_t)j * D + k0 + kq * 4);
-            sQ[kq * 4 + 0][r] = qv.x; sQ[kq * 4 + 1][r] = qv.y; sQ[kq * 4 + 2][r] = qv.z; sQ[kq * 4 + 3][r] = qv.w;
-            sC[kq * 4 + 0][r] = cv.x; sC[kq * 4 + 1][r] = cv.y; sC[kq * 4 + 2][r] = cv.z; sC[kq * 4 + 3][r] = cv.w;
+    for (int kc = 0; kc < D / kPK; ++kc) {
+        if (kc + 1 < D / kPK) {
+            load((kc + 1) * kPK, (kc + 1) & 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
         }
         __syncthreads();
-#pragma unroll 4
-        for (int k = 0; k < kPK; ++k) {
-            const float4 q0 = *reinterpret_cast<const float4 *>(&sQ[k][ty * 8]);
-            const float4 q1 = *reinterpret_cast<const float4 *>(&sQ[k][ty * 8 + 4]);
-            const float4 c0 = *reinterpret_cast<const float4 *>(&sC[k][tx * 8]);
-            const float4 c1 = *reinterpret_cast<const float4 *>(&sC[k][tx * 8 + 4]);
-            const float qr[8] = {q0.x, q0.y, q0.z, q0.w, q1.x, q1.y, q1.z, q1.w};
-            const float cr[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+        const float *sQ = psm + (kc & 1) * 2 * kPT * kPS;
+        const float *sC = sQ + kPT * kPS;
+#pragma unroll 1
+        for (int k = 0; k < kPK; k += 2) {
+            float2 qv[8], cv[8];
+#pragma unroll
+            for (int r = 0; r < 8; ++r) qv[r] = *reinterpret_cast<const float2 *>(sQ + (ty * 8 + r) * kPS + k);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) cv[c] = *reinterpret_cast<const float2 *>(sC + (tx + 16 * c) * kPS + k);
 #pragma unroll
             for (int r = 0; r < 8; ++r)
 #pragma unroll
-                for (int c = 0; c < 8; ++c) acc[r][c] = fmaf(qr[r], cr[c], acc[r][c]);
+                for (int c = 0; c < 8; ++c) {
+                    acc[r][c] = fmaf(qv[r].x, cv[c].x, acc[r][c]);
+                    acc[r][c] = fmaf(qv[r].y, cv[c].y, acc[r][c]);
+                }
         }
-        __syncthreads();
+        __syncthreads();   // this stage is refilled two chunks on
     }
+
     const float tc = QUANT ? 0.f : __ldg(a.tau_c + h);
     const float tr = QUANT ? 0.f : __ldg(a.tau_r + h);
     const size_t nP = (size_t)a.nB * (a.nB + 1) / 2;
@@ -221,38 +254,44 @@ __global__ void __launch_bounds__(256) k_pair_tile(const RbsArgs a)
     float rj[8];
 #pragma unroll
     for (int c = 0; c < 8; ++c) {
-        const int j = J * kPT + tx * 8 + c;
+        const int j = J * kPT + tx + 16 * c;
         rj[c] = j < a.nB ? a.rad[(size_t)g * a.nB + j] : 0.f;
     }
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
         const int i = I * kPT + ty * 8 + r;
         const float qn = i < a.nB ? a.qnorm[(size_t)h * a.nB + i] : 0.f;
-        uint32_t byte = 0;
+        bool keep[8];
 #pragma unroll
         for (int c = 0; c < 8; ++c) {
-            const int j = J * kPT + tx * 8 + c;
-            if (i >= a.nB || j > i) continue;
+            const int j = J * kPT + tx + 16 * c;
+            const bool valid = i < a.nB && j <= i;
             const float qc = acc[r][c];
             const float sc = a.scale * qc;
             const float sr = a.scale * fmaf(qn, rj[c], qc);
             if (QUANT) {
-                const size_t p = (size_t)i * (i + 1) / 2 + j;
-                a.pair_sc[(size_t)h * nP + p] = sc;
-                a.pair_sc[((size_t)a.Hq + h) * nP + p] = sr;
+                if (valid) {
+                    const size_t p = (size_t)i * (i + 1) / 2 + j;
+                    a.pair_sc[(size_t)h * nP + p] = sc;
+                    a.pair_sc[((size_t)a.Hq + h) * nP + p] = sr;
+                }
+                keep[c] = false;
             } else {
-                const bool keep = sc > tc || sr > tr || (a.force_diag && j == i) || (a.force_first && j == 0);
-                byte |= (uint32_t)keep << c;
+                keep[c] = valid && (sc > tc || sr > tr || (a.force_diag && j == i) || (a.force_first && j == 0));
             }
         }
         if (!QUANT) {
-            // word = 4 consecutive tx (32 columns); lanes tx..tx+3 are adjacent
-            uint32_t w = byte << ((tx & 3) * 8);
-            w |= __shfl_xor_sync(0xffffffffu, w, 1);
-            w |= __shfl_xor_sync(0xffffffffu, w, 2);
-            if ((tx & 3) == 0 && i < a.nB) {
-                a.bits[((size_t)h * a.nB + i) * words + J * 4 + (tx >> 2)] = w;
-                if (w) atomicAdd(&a.rowcnt[h * a.nB + i], __popc(w));
+            // word m of the row covers columns 32m + [0, 16) (cc = 2m, lanes tx)
+            // and 32m + [16, 32) (cc = 2m + 1); lanes 0-15 and 16-31 hold two rows
+#pragma unroll
+            for (int m = 0; m < 4; ++m) {
+                const unsigned b0 = __ballot_sync(0xffffffffu, keep[2 * m]);
+                const unsigned b1 = __ballot_sync(0xffffffffu, keep[2 * m + 1]);
+                const unsigned w = lane < 16 ? ((b0 & 0xffffu) | (b1 << 16)) : ((b0 >> 16) | (b1 & 0xffff0000u));
+                if ((lane & 15) == 0 && i < a.nB) {
+                    a.bits[((size_t)h * a.nB + i) * words + J * 4 + m] = w;
+                    if (w) atomicAdd(&a.rowcnt[h * a.nB + i], __popc(w));
+                }
             }
         }
     }
@@ -546,7 +585,11 @@ cudaError_t launch_rbs(const RbsArgs &a, cudaStream_t s)
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int nTB = (a.nB + kPT - 1) / kPT;
     const int tiles = nTB * (nTB + 1) / 2;
-    const size_t smem = 0;
+    const size_t smem = kPairSmem;
+    cudaError_t e0 = cudaFuncSetAttribute(k_pair_tile<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e0 == cudaSuccess)
+        e0 = cudaFuncSetAttribute(k_pair_tile<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e0 != cudaSuccess) return e0;
     if (quant) {
         if (cudaError_t e_ = launch_pdl(k_pair_tile<true>, dim3(dim3(tiles, a.Hq)), dim3(256), smem, s, a)) return e_;
         if ((e = cudaMemsetAsync(a.qhist, 0, (size_t)2 * a.Hq * (3 * 2048 + 4) * 4, s)) != cudaSuccess) return e;
