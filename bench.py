@@ -485,7 +485,11 @@ def tiered_measure(msk, cfg, dev, steps=64, slot_frac=0.125):
     m = cfg.msk
     P, L = m["P"], m["L"]
     n_pages = int(msk.cache.page_table.numel())
-    tier = T.TieredKV(msk.cache, slots=max(1, int(slot_frac * n_pages)), device=dev, time_fetches=True)
+    # at least three steps' pages (a focus step reads two chunks per sequence),
+    # since the pages of the step in flight stay resident
+    step_pages = m["B"] * (2 * 2048 // P + 1)
+    tier = T.TieredKV(msk.cache, slots=max(int(slot_frac * n_pages), 3 * step_pages), device=dev,
+                      time_fetches=True)
     V = DA.DAVocab()
     n_chunks = L // 2048
     machines = [DA.DAStateMachine(L - steps) for _ in range(m["B"])]
@@ -509,7 +513,7 @@ def tiered_measure(msk, cfg, dev, steps=64, slot_frac=0.125):
             mach.observe(tokens(i, b))
             lists.append(mach.next_spans(lens[b]))
         spans, cnt, rnd = SP.pack(lists, dev, max_spans=2)
-        tier.prepare([T.span_pages(l, n, P) for l, n in zip(lists, lens)])
+        tier.prepare([T.span_pages(l, n, P) for l, n in zip(lists, lens)], seq_lens=lens)
         c = tier.cache
         sel = sa.select_blocks_spans(c, spans, cnt, rnd, ws=ws)
         sa.sparse_decode_attn(c, msk.q_steps[i % msk.q_steps.shape[0]], sel, 1 / math.sqrt(m["d"]), 8,

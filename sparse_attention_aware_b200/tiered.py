@@ -115,7 +115,14 @@ class TieredKV:
         self.host_k = cache.k.cpu().pin_memory()
         self.host_v = cache.v.cpu().pin_memory()
         self.host_pt = cache.page_table.cpu().numpy().astype(np.int64)   # logical -> host page
-        self.seq_lens = cache.seq_lens.to(self.device)
+        # sequence lengths, published with the page table: two device copies
+        # used alternately (the step in flight keeps reading its own), each
+        # filled from a pinned mirror on the copy stream
+        lens0 = cache.seq_lens.to(torch.int32).cpu()
+        self.dev_lens = [lens0.to(self.device), lens0.to(self.device)]
+        self.lens_mirror = [lens0.clone().pin_memory() for _ in range(2)]
+        self.lens_free = [None, None]
+        self.lens_cur = 0
         self.map = SlotMap(self.host_k.shape[0], slots)
         shape = (slots,) + tuple(self.host_k.shape[1:])
         self.dev_k = torch.zeros(shape, dtype=torch.bfloat16, device=self.device)
@@ -147,7 +154,11 @@ class TieredKV:
     @property
     def cache(self) -> PagedCache:
         """The device view: slot pools and the published page table."""
-        return PagedCache(self.dev_k, self.dev_v, self.dev_pt, self.seq_lens)
+        return PagedCache(self.dev_k, self.dev_v, self.dev_pt, self.dev_lens[self.lens_cur])
+
+    @property
+    def seq_lens(self) -> torch.Tensor:
+        return self.dev_lens[self.lens_cur]
 
     def page_bytes(self) -> int:
         return self.host_k[0].numel() * 2
@@ -156,11 +167,19 @@ class TieredKV:
         parts = [self.host_pt[b, np.asarray(pages, dtype=np.int64)] for b, pages in enumerate(need) if len(pages)]
         return np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
 
-    def prepare(self, need: Sequence[Iterable[int]], compute_stream: Optional[torch.cuda.Stream] = None) -> int:
+    def prepare(self, need: Sequence[Iterable[int]], compute_stream: Optional[torch.cuda.Stream] = None,
+                seq_lens: Optional[Sequence[int]] = None) -> int:
         """Make the logical pages ``need[b]`` of every sequence resident:
         fetch the missing ones and publish the page table on the copy stream;
         the compute stream waits for both before its next launch.  Returns the
-        number of pages fetched."""
+        number of pages fetched.
+
+        ``seq_lens`` (one per sequence) are published with the table and
+        become ``cache.seq_lens`` for the step.  The span and top-k kernels clip
+        what they read to these lengths, so ``need`` must be computed with the
+        same ones (``span_pages(spans, seq_lens[b], P)``): a span that reaches
+        past the length the host clipped to would make the device read a page
+        that was never requested."""
         compute_stream = compute_stream or torch.cuda.current_stream(self.device)
         # the step queued just before this call may still be running and its
         # pages are kept; older steps must be done before a slot is reused
@@ -174,6 +193,13 @@ class TieredKV:
         if pairs:
             pa = np.asarray(pairs)
             self.pt[self.where_b[pa[:, 0]], self.where_lp[pa[:, 0]]] = pa[:, 1]
+        lbuf = self.lens_cur ^ 1
+        if seq_lens is not None:
+            if len(seq_lens) != self.host_pt.shape[0]:
+                raise ValueError("seq_lens: one length per sequence")
+            if self.lens_free[lbuf] is not None:
+                self.lens_free[lbuf].synchronize()
+            self.lens_mirror[lbuf].numpy()[...] = np.asarray(seq_lens, dtype=np.int32)
         buf = self.flip
         if changed:
             self.flip ^= 1
@@ -199,7 +225,16 @@ class TieredKV:
                 done = torch.cuda.Event()
                 done.record(self.stream)
                 self.mirror_free[buf] = done
+            if seq_lens is not None:
+                # the buffer last served the step before the one in flight,
+                # which prev_mark orders before this copy
+                self.dev_lens[lbuf].copy_(self.lens_mirror[lbuf], non_blocking=True)
+                done = torch.cuda.Event()
+                done.record(self.stream)
+                self.lens_free[lbuf] = done
             self.ready.record(self.stream)
         compute_stream.wait_event(self.ready)
+        if seq_lens is not None:
+            self.lens_cur = lbuf
         self.prev_mark = mark
         return len(pairs)

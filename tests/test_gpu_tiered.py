@@ -45,22 +45,25 @@ def test_fetch_pages_copies_whole_pages_and_records_bad_pairs(cuda_dev):
 
 
 def test_tiered_masked_decode_is_bitwise_the_resident_decode(cuda_dev):
-    """A DA tag stream over 3 sequences with a device pool of ~40% of the
-    pages: every step's block list and decode equal those of the fully
-    resident cache bit for bit, and the oracle agrees."""
+    """A DA tag stream over 3 sequences with a device pool of half of the
+    pages and lengths published by the tier each step: every step's block
+    list and decode equal those of the fully resident cache bit for bit, and
+    the oracle agrees."""
     V = DA.DAVocab()
     G, LOC, FO, FC = V.global_tag, V.local_tag, V.focus_open, V.focus_close
     C = lambda c: V.chunk_base + c
     P, Hq, Hkv, d = 16, 16, 2, 128
-    prompts = [12000, 9000, 10000]
-    streams = [[LOC, FO, C(1), C(4), FC, 3, FO, C(0), FC, LOC, 5, FO, C(2), FC],
+    # sequence 0's first focus chunk (5) runs past its decode length: the
+    # pages past the length are neither requested nor read
+    prompts = [11990, 9000, 10000]
+    streams = [[LOC, FO, C(5), FC, FO, C(1), C(4), FC, 3, FO, C(0), FC, LOC, 5],
                [FO, C(2), FC, 1, LOC, 2, FO, C(3), C(1), FC, 4, 5, LOC, 6],
                [LOC, 1, 2, FO, C(0), C(3), FC, 3, 4, LOC, FO, C(4), FC, 7]]
     steps = len(streams[0])
     cap = [L + steps for L in prompts]
     full, _ = W.random_decode(77, 3, Hq, Hkv, d, cap, P)
     pages_total = sum((L + P - 1) // P for L in cap)
-    tier = T.TieredKV(full, slots=int(0.4 * pages_total), device=cuda_dev)
+    tier = T.TieredKV(full, slots=int(0.5 * pages_total), device=cuda_dev)
     res = full.to(cuda_dev)
     machine = DA.DABatch(prompts)
     ws_t, ws_r = sa.Workspace(cuda_dev), sa.Workspace(cuda_dev)
@@ -75,8 +78,9 @@ def test_tiered_masked_decode_is_bitwise_the_resident_decode(cuda_dev):
             m.observe(streams[b][i])
             lists.append(m.next_spans(lens[b]))
         spans, cnt, rnd = SP.pack(lists, cuda_dev, max_spans=2)
-        fetched += tier.prepare([T.span_pages(l, L, P) for l, L in zip(lists, lens)])
-        tc = W.PagedCache(tier.dev_k, tier.dev_v, tier.dev_pt, lens_t)
+        fetched += tier.prepare([T.span_pages(l, L, P) for l, L in zip(lists, lens)], seq_lens=lens)
+        tc = tier.cache
+        assert torch.equal(tc.seq_lens, lens_t)
         rc = W.PagedCache(res.k, res.v, res.page_table, lens_t)
         sel_t = sa.select_blocks_spans(tc, spans, cnt, rnd, ws=ws_t)
         sel_r = sa.select_blocks_spans(rc, spans, cnt, rnd, ws=ws_r)
