@@ -10,36 +10,35 @@
 // Kernels (one launch sequence per call):
 //   k_block_stats  per (key block j, kv head g): c_j = mean of the block's keys,
 //                  r_j = max ||k - c_j||, from one read of the block (staged in
-//                  shared memory).
+//                  shared memory); c_j is written as a split-bf16 tile image
+//                  for the tensor cores.
 //   k_pool_q       per (query block i, q head h): qbar_i = mean of the block's
-//                  queries, ||qbar_i||.
-//   k_pair_tile    per (128x128 tile of causal block pairs, q head): the pooled
-//                  dot products qbar_i . c_j (fp32 SIMT tile product), both
-//                  branch scores, thresholds, OR with the forced diagonal and
-//                  first block -> mask bits and per-row counts.  In quantile
-//                  mode the scores are stored instead and
+//                  queries (tile image, as c_j), ||qbar_i||.
+//   k_pair_tc      (k_pair_tc.cu) per (128-block row tile, q head) on tcgen05:
+//                  the pooled dot products qbar_i . c_j, both branch scores,
+//                  thresholds, OR with the forced diagonal and first block ->
+//                  mask bits and per-row counts.  In quantile mode the scores
+//                  are stored instead and
 //   k_qhist/k_qpick  find each head's lower quantile (exact radix select on
 //                  the order-preserving key, grid-wide histograms) and
 //   k_mask_scores  thresholds the stored scores.
 //   k_csr_scan / k_csr_fill  turn counts and bits into CSR (ascending cols).
+#include <cuda_bf16.h>
+
 #include "sa_internal.h"
 
 namespace sa {
 
-namespace {
-// mask bit words per (head, query block) row: 4 per 128-wide tile column
-__host__ __device__ inline int mask_words(int nB) { return 4 * ((nB + 127) / 128); }
-}  // namespace
-
 size_t rbs_workspace_layout(int Hq, int Hkv, int D, int nB, bool quantile, size_t *offs)
 {
     auto up = [](size_t x) { return (x + 255) / 256 * 256; };
-    const size_t words = mask_words(nB);
+    const size_t words = rbs_mask_words(nB);
     const size_t nP = (size_t)nB * (nB + 1) / 2;
     size_t o = 0;
-    offs[0] = o; o += up((size_t)Hkv * nB * D * 4);       // centroids
+    const size_t img = (size_t)rbs_img_tiles(nB) * kRbsImgBytes;   // per matrix (D = 128)
+    offs[0] = o; o += up((size_t)Hkv * img);              // centroid tile images
     offs[1] = o; o += up((size_t)Hkv * nB * 4);           // radii
-    offs[2] = o; o += up((size_t)Hq * nB * D * 4);        // pooled queries
+    offs[2] = o; o += up((size_t)Hq * img);               // pooled-query tile images
     offs[3] = o; o += up((size_t)Hq * nB * 4);            // pooled query norms
     offs[4] = o; o += up((size_t)2 * Hq * 4);             // thresholds
     offs[5] = o; o += up((size_t)Hq * nB * words * 4);    // mask bits
@@ -55,6 +54,15 @@ namespace {
 
 constexpr int BS = 64;   // block size (tokens); query and key blocks alike
 
+// x -> (hi, lo) = (bf16(x), bf16(x - hi)) at element (row, k) of a tile image
+__device__ __forceinline__ void store_split(uint8_t *img, int row, int k, float x)
+{
+    const __nv_bfloat16 hi = __float2bfloat16_rn(x);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(x - __bfloat162float(hi));
+    *reinterpret_cast<__nv_bfloat16 *>(img + rbs_img_offset(row, k, 0)) = hi;
+    *reinterpret_cast<__nv_bfloat16 *>(img + rbs_img_offset(row, k, 1)) = lo;
+}
+
 // ---------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) k_block_stats(const RbsArgs a)
 {
@@ -65,6 +73,14 @@ __global__ void __launch_bounds__(256) k_block_stats(const RbsArgs a)
     __shared__ float cen[D];
     __shared__ float wmax[8];
     const int j = blockIdx.x, g = blockIdx.y;
+    uint8_t *img = a.cen + ((size_t)g * rbs_img_tiles(a.nB) + (j >> 7)) * kRbsImgBytes;
+    if (j >= a.nB) {   // padding row of the last tile image
+        if (threadIdx.x < D) {
+            *reinterpret_cast<uint16_t *>(img + rbs_img_offset(j & 127, threadIdx.x, 0)) = 0;
+            *reinterpret_cast<uint16_t *>(img + rbs_img_offset(j & 127, threadIdx.x, 1)) = 0;
+        }
+        return;
+    }
     const int n = min(BS, a.T - j * BS);
     const int P = 1 << a.c.Plog2;
     // stage the block's rows (16-byte chunks; 16 per row)
@@ -87,7 +103,7 @@ __global__ void __launch_bounds__(256) k_block_stats(const RbsArgs a)
         for (int r = 0; r < n; ++r) s += __uint_as_float((uint32_t)tile[r * D + threadIdx.x] << 16);
         const float c = s / (float)n;
         cen[threadIdx.x] = c;
-        a.cen[((size_t)g * a.nB + j) * D + threadIdx.x] = c;
+        store_split(img, j & 127, threadIdx.x, c);
     }
     __syncthreads();
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -121,6 +137,14 @@ __global__ void __launch_bounds__(256) k_pool_q(const RbsArgs a)
     __shared__ float part[16][D];
     __shared__ float red[4];
     const int i = blockIdx.x, h = blockIdx.y;
+    uint8_t *img = a.qbar + ((size_t)h * rbs_img_tiles(a.nB) + (i >> 7)) * kRbsImgBytes;
+    if (i >= a.nB) {   // padding row of the last tile image
+        if (threadIdx.x < D) {
+            *reinterpret_cast<uint16_t *>(img + rbs_img_offset(i & 127, threadIdx.x, 0)) = 0;
+            *reinterpret_cast<uint16_t *>(img + rbs_img_offset(i & 127, threadIdx.x, 1)) = 0;
+        }
+        return;
+    }
     const int n = min(BS, a.T - i * BS);
     const int lane16 = threadIdx.x & 15, rs = threadIdx.x >> 4;   // 16 row slots
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -139,162 +163,13 @@ __global__ void __launch_bounds__(256) k_pool_q(const RbsArgs a)
 #pragma unroll
         for (int r = 0; r < 16; ++r) s += part[r][threadIdx.x];
         const float qb = s / (float)n;
-        a.qbar[((size_t)h * a.nB + i) * D + threadIdx.x] = qb;
+        store_split(img, i & 127, threadIdx.x, qb);
         sq = qb * qb;
     }
     sq = warp_sum(sq);
     if ((threadIdx.x & 31) == 0 && threadIdx.x < D) red[threadIdx.x >> 5] = sq;
     __syncthreads();
     if (threadIdx.x == 0) a.qnorm[(size_t)h * a.nB + i] = sqrtf((red[0] + red[1]) + (red[2] + red[3]));
-}
-
-// ---------------------------------------------------------------------------
-// lower-triangular tile index -> (I, J), J <= I
-__device__ __forceinline__ void tri_index(int x, int &I, int &J)
-{
-    int r = (int)((sqrtf(8.f * (float)x + 1.f) - 1.f) * 0.5f);
-    while ((r + 1) * (r + 2) / 2 <= x) ++r;
-    while (r * (r + 1) / 2 > x) --r;
-    I = r;
-    J = x - r * (r + 1) / 2;
-}
-
-// 128 x 128 tile of causal block pairs of one head: qbar_i . c_j for i in the
-// row tile I, j in the column tile J <= I (fp32 SIMT: 256 threads, 8 x 8
-// outputs each, K staged through shared memory in chunks of 32, transposed so
-// each thread reads its 8 rows and 8 columns with two 16-byte loads each).
-constexpr int kPT = 128;   // tile edge (blocks)
-constexpr int kPK = 32;    // K chunk
-
-constexpr int kPS = kPK + 2;   // shared row stride (floats): 8-byte column reads hit 32 distinct banks
-constexpr int kPairSmem = 2 * 2 * kPT * kPS * 4;   // 2 stages x (qbar, c) chunks
-
-__device__ __forceinline__ void cp_async8(uint32_t dst, const void *src, bool pred)
-{
-    asm volatile("cp.async.ca.shared.global [%0], [%1], 8, %2;" ::"r"(dst), "l"(src), "r"(pred ? 8 : 0)
-                 : "memory");
-}
-
-// Pooled dot products of one 128x128 tile of (query block, key block) pairs:
-// 32-wide chunks of d stream into a double-buffered shared-memory tile with
-// cp.async (rows padded to kPS floats), each thread accumulating 8 query
-// rows x 8 key columns (columns tx + 16*cc, so a warp's 8-byte column reads
-// cover all banks once) in ascending d order.
-template <bool QUANT>
-__global__ void __launch_bounds__(256, 2) k_pair_tile(const RbsArgs a)
-{
-    pdl_wait();
-    pdl_trigger();
-    constexpr int D = 128;
-    extern __shared__ __align__(16) float psm[];
-    int I, J;
-    tri_index(blockIdx.x, I, J);
-    const int h = blockIdx.y;
-    const int g = h / (a.Hq / a.c.Hkv);
-    const int tid = threadIdx.x, lane = tid & 31;
-    const int ty = tid >> 4, tx = tid & 15;
-    const float *qb = a.qbar + (size_t)h * a.nB * D;
-    const float *cb = a.cen + (size_t)g * a.nB * D;
-    const uint32_t sb = (uint32_t)__cvta_generic_to_shared(psm);
-
-    // chunk k0 of both operands into stage st: 128 rows x 16 pieces of 8 bytes each
-    auto load = [&](int k0, int st) {
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-            const int x = tid + 256 * u;
-            const int r = x >> 4, pc = x & 15;
-            const int i = I * kPT + r, j = J * kPT + r;
-            const uint32_t off = (uint32_t)((st * 2 * kPT + r) * kPS + pc * 2) * 4;
-            cp_async8(sb + off, qb + (size_t)(i < a.nB ? i : 0) * D + k0 + pc * 2, i < a.nB);
-            cp_async8(sb + off + kPT * kPS * 4, cb + (size_t)(j < a.nB ? j : 0) * D + k0 + pc * 2, j < a.nB);
-        }
-        asm volatile("cp.async.commit_group;" ::: "memory");
-    };
-
-    float acc[8][8];
-#pragma unroll
-    for (int r = 0; r < 8; ++r)
-#pragma unroll
-        for (int c = 0; c < 8; ++c) acc[r][c] = 0.f;
-
-    load(0, 0);
-#pragma unroll 1
-    for (int kc = 0; kc < D / kPK; ++kc) {
-        if (kc + 1 < D / kPK) {
-            load((kc + 1) * kPK, (kc + 1) & 1);
-            asm volatile("cp.async.wait_group 1;" ::: "memory");
-        } else {
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
-        }
-        __syncthreads();
-        const float *sQ = psm + (kc & 1) * 2 * kPT * kPS;
-        const float *sC = sQ + kPT * kPS;
-#pragma unroll 1
-        for (int k = 0; k < kPK; k += 2) {
-            float2 qv[8], cv[8];
-#pragma unroll
-            for (int r = 0; r < 8; ++r) qv[r] = *reinterpret_cast<const float2 *>(sQ + (ty * 8 + r) * kPS + k);
-#pragma unroll
-            for (int c = 0; c < 8; ++c) cv[c] = *reinterpret_cast<const float2 *>(sC + (tx + 16 * c) * kPS + k);
-#pragma unroll
-            for (int r = 0; r < 8; ++r)
-#pragma unroll
-                for (int c = 0; c < 8; ++c) {
-                    acc[r][c] = fmaf(qv[r].x, cv[c].x, acc[r][c]);
-                    acc[r][c] = fmaf(qv[r].y, cv[c].y, acc[r][c]);
-                }
-        }
-        __syncthreads();   // this stage is refilled two chunks on
-    }
-
-    const float tc = QUANT ? 0.f : __ldg(a.tau_c + h);
-    const float tr = QUANT ? 0.f : __ldg(a.tau_r + h);
-    const size_t nP = (size_t)a.nB * (a.nB + 1) / 2;
-    const int words = mask_words(a.nB);
-    float rj[8];
-#pragma unroll
-    for (int c = 0; c < 8; ++c) {
-        const int j = J * kPT + tx + 16 * c;
-        rj[c] = j < a.nB ? a.rad[(size_t)g * a.nB + j] : 0.f;
-    }
-#pragma unroll
-    for (int r = 0; r < 8; ++r) {
-        const int i = I * kPT + ty * 8 + r;
-        const float qn = i < a.nB ? a.qnorm[(size_t)h * a.nB + i] : 0.f;
-        bool keep[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-            const int j = J * kPT + tx + 16 * c;
-            const bool valid = i < a.nB && j <= i;
-            const float qc = acc[r][c];
-            const float sc = a.scale * qc;
-            const float sr = a.scale * fmaf(qn, rj[c], qc);
-            if (QUANT) {
-                if (valid) {
-                    const size_t p = (size_t)i * (i + 1) / 2 + j;
-                    a.pair_sc[(size_t)h * nP + p] = sc;
-                    a.pair_sc[((size_t)a.Hq + h) * nP + p] = sr;
-                }
-                keep[c] = false;
-            } else {
-                keep[c] = valid && (sc > tc || sr > tr || (a.force_diag && j == i) || (a.force_first && j == 0));
-            }
-        }
-        if (!QUANT) {
-            // word m of the row covers columns 32m + [0, 16) (cc = 2m, lanes tx)
-            // and 32m + [16, 32) (cc = 2m + 1); lanes 0-15 and 16-31 hold two rows
-#pragma unroll
-            for (int m = 0; m < 4; ++m) {
-                const unsigned b0 = __ballot_sync(0xffffffffu, keep[2 * m]);
-                const unsigned b1 = __ballot_sync(0xffffffffu, keep[2 * m + 1]);
-                const unsigned w = lane < 16 ? ((b0 & 0xffffu) | (b1 << 16)) : ((b0 >> 16) | (b1 & 0xffff0000u));
-                if ((lane & 15) == 0 && i < a.nB) {
-                    a.bits[((size_t)h * a.nB + i) * words + J * 4 + m] = w;
-                    if (w) atomicAdd(&a.rowcnt[h * a.nB + i], __popc(w));
-                }
-            }
-        }
-    }
 }
 
 // ---------------------------------------------------------------------------
@@ -447,7 +322,7 @@ __global__ void __launch_bounds__(256) k_mask_scores(const RbsArgs a)
     const float *sc = a.pair_sc + (size_t)h * nP + (size_t)i * (i + 1) / 2;
     const float *sr = a.pair_sc + ((size_t)a.Hq + h) * nP + (size_t)i * (i + 1) / 2;
     const float tc = a.tau[h], tr = a.tau[a.Hq + h];
-    const int words = mask_words(a.nB);
+    const int words = rbs_mask_words(a.nB);
     const int nw = i / 32 + 1;
     int cnt = 0;
     for (int w0 = 0; w0 < nw; w0 += 4) {
@@ -528,7 +403,7 @@ __global__ void __launch_bounds__(256) k_csr_fill(const RbsArgs a)
     const int lane = threadIdx.x & 31;
     if (row >= a.Hq * a.nB) return;
     const int i = row % a.nB;
-    const int words = mask_words(a.nB);
+    const int words = rbs_mask_words(a.nB);
     const int nw = i / 32 + 1;
     long long base = a.row_ptr[row];
     for (int w0 = 0; w0 < nw; w0 += 32) {
@@ -580,18 +455,12 @@ cudaError_t launch_rbs(const RbsArgs &a, cudaStream_t s)
     const bool quant = a.tau_c == nullptr;
     cudaError_t e;
     // per-kv-head block statistics on sequence 0's keys
-    if (cudaError_t e_ = launch_pdl(k_block_stats, dim3(dim3(a.nB, a.c.Hkv)), dim3(256), 0, s, a)) return e_;
-    if (cudaError_t e_ = launch_pdl(k_pool_q, dim3(dim3(a.nB, a.Hq)), dim3(256), 0, s, a)) return e_;
+    const int img_rows = rbs_img_tiles(a.nB) * kRbsImgRows;   // padding rows are zeroed
+    if (cudaError_t e_ = launch_pdl(k_block_stats, dim3(dim3(img_rows, a.c.Hkv)), dim3(256), 0, s, a)) return e_;
+    if (cudaError_t e_ = launch_pdl(k_pool_q, dim3(dim3(img_rows, a.Hq)), dim3(256), 0, s, a)) return e_;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const int nTB = (a.nB + kPT - 1) / kPT;
-    const int tiles = nTB * (nTB + 1) / 2;
-    const size_t smem = kPairSmem;
-    cudaError_t e0 = cudaFuncSetAttribute(k_pair_tile<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e0 == cudaSuccess)
-        e0 = cudaFuncSetAttribute(k_pair_tile<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e0 != cudaSuccess) return e0;
     if (quant) {
-        if (cudaError_t e_ = launch_pdl(k_pair_tile<true>, dim3(dim3(tiles, a.Hq)), dim3(256), smem, s, a)) return e_;
+        if ((e = launch_pair_tc(a, true, s)) != cudaSuccess) return e;
         if ((e = cudaMemsetAsync(a.qhist, 0, (size_t)2 * a.Hq * (3 * 2048 + 4) * 4, s)) != cudaSuccess) return e;
         const size_t nP = (size_t)a.nB * (a.nB + 1) / 2;
         const dim3 hgrid((unsigned)((nP + kQChunk - 1) / kQChunk), 2 * a.Hq);
@@ -603,7 +472,7 @@ cudaError_t launch_rbs(const RbsArgs &a, cudaStream_t s)
     } else {
         if (cudaError_t e_ = launch_pdl(k_copy_tau, dim3((a.Hq + 127) / 128), dim3(128), 0, s, a)) return e_;
         if ((e = cudaMemsetAsync(a.rowcnt, 0, (size_t)a.Hq * a.nB * sizeof(int32_t), s)) != cudaSuccess) return e;
-        if (cudaError_t e_ = launch_pdl(k_pair_tile<false>, dim3(dim3(tiles, a.Hq)), dim3(256), smem, s, a)) return e_;
+        if ((e = launch_pair_tc(a, false, s)) != cudaSuccess) return e;
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     {

@@ -340,13 +340,12 @@ sa_status sa_select_blocks(const sa_kv_cache *kv, const sa_block_select_args *ar
     a.p_r = args->p_r;
     a.force_diag = args->force_diag;
     a.force_first = args->force_first;
-    a.cen = reinterpret_cast<float *>(w + offs[0]);
+    a.cen = reinterpret_cast<uint8_t *>(w + offs[0]);
     a.rad = reinterpret_cast<float *>(w + offs[1]);
-    a.qbar = reinterpret_cast<float *>(w + offs[2]);
+    a.qbar = reinterpret_cast<uint8_t *>(w + offs[2]);
     a.qnorm = reinterpret_cast<float *>(w + offs[3]);
     a.tau = reinterpret_cast<float *>(w + offs[4]);
     a.bits = reinterpret_cast<uint32_t *>(w + offs[5]);
-    a.words = (nB + 31) / 32;
     a.rowcnt = reinterpret_cast<int32_t *>(w + offs[6]);
     a.pair_sc = quant ? reinterpret_cast<float *>(w + offs[7]) : nullptr;
     a.qhist = quant ? reinterpret_cast<uint32_t *>(w + offs[8]) : nullptr;

@@ -96,13 +96,12 @@ struct RbsArgs {
     float p_c, p_r;
     int force_diag, force_first;
     // workspace pieces
-    float *cen;      // [Hkv][nB][D]
+    uint8_t *cen;    // centroids, tile images [Hkv][nTB][64 KB] (rbs_img_offset)
     float *rad;      // [Hkv][nB]
-    float *qbar;     // [Hq][nB][D]
+    uint8_t *qbar;   // pooled queries, tile images [Hq][nTB][64 KB]
     float *qnorm;    // [Hq][nB]
     float *tau;      // [2][Hq] thresholds in use
-    uint32_t *bits;  // [Hq][nB][nB/32 words] mask bits
-    int words;       // words per row
+    uint32_t *bits;  // [Hq][nB][rbs_mask_words(nB)] mask bits
     int32_t *rowcnt; // [Hq*nB]
     float *pair_sc;  // quantile mode: [Hq][nP] S_c, [Hq][nP] S_r
     uint32_t *qhist; // quantile mode scratch
@@ -113,8 +112,26 @@ struct RbsArgs {
     float *tau_out;
     DevStatus *st;
 };
+// mask bit words per (head, query block) row: 4 per 128-wide column tile
+__host__ __device__ inline int rbs_mask_words(int nB) { return 4 * ((nB + 127) / 128); }
+// Pooled vectors (d = 128) as tensor-core tile images: each fp32 value x is
+// kept as two bf16 parts, hi = bf16(x) and lo = bf16(x - hi); 128 blocks form
+// a 64 KB tile [part][K half][row][128 bytes] in the 128-byte-swizzled K-major
+// layout (16-byte chunk c of a row's K half stored at chunk c ^ (row % 8)).
+// Tile t of matrix m (a head or kv head) starts at (m * nTB + t) * 64 KB.
+constexpr int kRbsImgRows = 128;
+constexpr uint32_t kRbsImgBytes = 65536;
+__host__ __device__ inline int rbs_img_tiles(int nB) { return (nB + kRbsImgRows - 1) / kRbsImgRows; }
+__host__ __device__ inline uint32_t rbs_img_offset(int row, int k, int part)
+{
+    return (uint32_t)(part * 2 + (k >> 6)) * 16384u + (uint32_t)row * 128u +
+           ((uint32_t)(((k & 63) >> 3) ^ (row & 7)) << 4) + (uint32_t)(k & 7) * 2u;
+}
 size_t rbs_workspace_layout(int Hq, int Hkv, int D, int nB, bool quantile, size_t *offs);
 cudaError_t launch_rbs(const RbsArgs &a, cudaStream_t s);
+// pair scores + thresholds + OR + forced blocks on tcgen05 (mask words and
+// row counts; in quantile mode the two scores of every causal pair)
+cudaError_t launch_pair_tc(const RbsArgs &a, bool quant, cudaStream_t s);
 
 // ---- prefill ------------------------------------------------------------------
 struct PrefillArgs {
