@@ -168,6 +168,13 @@ typedef enum { SA_SEL_RBS = 1, SA_SEL_SPANS = 2 } sa_select_mode;
  *   for j <= i.  Thresholds: explicit per head (tau_c, tau_r: device fp32
  *   [num_q_heads]) or, when tau_c == NULL, the lower quantile p of the head's
  *   causal pair scores: sorted_asc[floor(p*(n-1))] (p_c, p_r).
+ *   scale must be finite and > 0 (SA_ERR_INVALID_ARGUMENT otherwise).
+ *   Precision: the products qbar_i . c_j run on tensor cores with each fp32
+ *   operand split into bf16 hi + lo parts (lo.hi + hi.lo + hi.hi, fp32
+ *   accumulation): |error| <= 3 * 2^-18 * scale * sum_k |qbar_ik c_jk| plus
+ *   fp32 rounding.  Explicit thresholds are applied as qbar.c > tau_c / scale
+ *   and qbar.c + ||qbar|| r > tau_r / scale (the same test up to fp32
+ *   rounding of the quotients).
  *   q          bf16 [num_tokens][num_q_heads][head_dim]
  *   Output: CSR over rows (h, i), row = h * nQB + i, nQB = ceil(T / block_size):
  *     row_ptr int32 [num_q_heads*nQB + 1], cols int32 [nnz_capacity] ascending.

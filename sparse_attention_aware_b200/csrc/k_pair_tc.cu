@@ -25,17 +25,19 @@
 // tiles J = 0..I.
 //   warp 8     producer and MMA issuer (one thread): bulk copies of the
 //              row's query tile image (once) and of each column's centroid
-//              image into a 2-stage ring; per column 24 MMAs (M = N = 128,
-//              K = 16: lo.hi, hi.lo, hi.hi per K step) into one of two TMEM
-//              accumulators, committed to that accumulator's mbarrier; a
-//              stage is refilled as soon as the MMAs that read it complete.
+//              image and radii into a 2-stage ring; per column 24 MMAs
+//              (M = N = 128, K = 16: lo.hi, hi.lo, hi.hi per K step) into
+//              one of two TMEM accumulators, committed to that accumulator's
+//              mbarrier; a stage is refilled as soon as the MMAs that read
+//              it complete.
 //   warps 0-7  epilogue: warp w reads TMEM lanes 32 (w % 4).. (its query
-//              blocks) and columns 64 (w / 4).. of the accumulator, frees it
-//              for the MMAs two columns on, then forms both branch scores,
-//              the thresholds and the OR (causal and forced blocks only in
-//              the first and diagonal column tiles) -> one 32-bit mask word
-//              per 32 columns, or in quantile mode stores the two scores.
-//              Per-row kept counts are summed over the row and added once.
+//              blocks) and columns 64 (w / 4).. of the accumulator and forms
+//              the thresholded branch scores and their OR as one 32-bit mask
+//              word per 32 columns (causal and forced bits applied per word
+//              in the first and diagonal column tiles), or in quantile mode
+//              stores the two scores; it then frees the accumulator for the
+//              MMAs two columns on.  Per-row kept counts are summed over the
+//              row and added once.
 // Waits are bounded (globaltimer deadline, shared abort flag); on expiry the
 // kernel records SA_ERR_TIMEOUT, every role leaves its loop, the producer
 // waits (bounded) for its outstanding copies and MMAs, TMEM is freed and the
@@ -55,9 +57,14 @@ constexpr int kThr = kEpiThreads + 32;        // + producer warp
 constexpr uint32_t kOp = kRbsImgBytes / 2;    // one part (hi or lo) of a tile image: 32 KB
 constexpr uint32_t kPiece = 16384;            // bulk-copy piece
 
+constexpr int kRadStages = 4;                 // radii ring (see the producer's refill rule)
+constexpr int kStgStride = 17;                // quantile-mode staging row stride (floats)
+
 constexpr uint32_t OFF_A = 0;                           // query tile image (hi, lo)
 constexpr uint32_t OFF_B = OFF_A + kRbsImgBytes;        // 2 stages of centroid tile images
-constexpr uint32_t OFF_BAR = OFF_B + 2 * kRbsImgBytes;  // a_full, b_full[2], mma_done[2], acc_free[2], drain
+constexpr uint32_t OFF_RAD = OFF_B + 2 * kRbsImgBytes;  // radii ring [kRadStages][kT]
+constexpr uint32_t OFF_STG = OFF_RAD + kRadStages * kT * 4;   // per epilogue warp: 32 x 16 scores
+constexpr uint32_t OFF_BAR = OFF_STG + 8 * 32 * kStgStride * 4;   // a_full, b_full[2], mma_done[2], acc_free[2], drain
 constexpr int kNumBars = 8;
 constexpr uint32_t OFF_MISC = OFF_BAR + kNumBars * 8;   // TMEM base, abort flag
 constexpr uint32_t kSmem = OFF_MISC + 8 + 1024;         // + slack for the 1024-byte alignment
@@ -70,11 +77,14 @@ __device__ __forceinline__ uint64_t op_desc(uint32_t base, int kk)
     return smem_desc_sw128(base + (uint32_t)(kk >> 2) * (kOp / 2) + (uint32_t)(kk & 3) * 32, 16, 1024);
 }
 
-__device__ __forceinline__ void load_image(uint8_t *dst, const uint8_t *src, uint64_t *bar)
+// one column tile: its centroid image and its 128 radii, on one barrier
+__device__ __forceinline__ void load_column(uint8_t *dst, const uint8_t *src, float *rad_dst, const float *rad_src,
+                                           uint64_t *bar)
 {
-    mbar_arrive_expect_tx(bar, kRbsImgBytes);
+    mbar_arrive_expect_tx(bar, kRbsImgBytes + kT * 4);
 #pragma unroll
     for (int q = 0; q < (int)(kRbsImgBytes / kPiece); ++q) bulk_load(dst + q * kPiece, src + q * kPiece, kPiece, bar);
+    bulk_load(rad_dst, rad_src, kT * 4, bar);
 }
 
 __device__ __forceinline__ float2 fmul2(float2 a, float2 b)
@@ -101,6 +111,8 @@ __global__ void __launch_bounds__(kThr, 1) k_pair_tc(const RbsArgs a, int nTB)
     uint64_t *a_full = bars, *b_full = bars + 1, *mma_done = bars + 3, *acc_free = bars + 5, *drain = bars + 7;
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + OFF_MISC);
     volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + OFF_MISC + 4);
+    float *srad = reinterpret_cast<float *>(smem + OFF_RAD);
+    const int rad_rows = nTB * kT;
 
     if (tid == 0) {
         mbar_init(a_full, 1);
@@ -125,13 +137,23 @@ __global__ void __launch_bounds__(kThr, 1) k_pair_tc(const RbsArgs a, int nTB)
         if (lane == 0) {
             const uint8_t *qimg = a.qbar + ((size_t)h * nTB + I) * kRbsImgBytes;
             const uint8_t *cimg = a.cen + (size_t)g * nTB * kRbsImgBytes;
-            int loads[2] = {0, 0}, waited[2] = {0, 0};   // centroid copies issued / consumed per stage
+            const float *radg = a.rad + (size_t)g * rad_rows;
+            int loads[2] = {0, 0}, waited[2] = {0, 0};   // column copies issued / consumed per stage
             bool a_pending = true;
-            load_image(smem + OFF_A, qimg, a_full);
-            for (int J = 0; J <= I && J < 2; ++J) {
-                load_image(smem + OFF_B + J * kRbsImgBytes, cimg + (size_t)J * kRbsImgBytes, b_full + J);
-                ++loads[J];
-            }
+            mbar_arrive_expect_tx(a_full, kRbsImgBytes);
+            for (int q = 0; q < (int)(kRbsImgBytes / kPiece); ++q)
+                bulk_load(smem + OFF_A + q * kPiece, qimg + q * kPiece, kPiece, a_full);
+            // Column J goes to image stage J % 2 and radii stage J % 4.  It is
+            // loaded after the MMAs of column J - 2 complete (the last reader
+            // of its image stage); those MMAs were issued after the epilogue
+            // of column J - 4 released its accumulator, so the radii stage of
+            // column J - 4 is free as well.
+            auto load_col = [&](int J) {
+                load_column(smem + OFF_B + (J & 1) * kRbsImgBytes, cimg + (size_t)J * kRbsImgBytes,
+                            srad + (J % kRadStages) * kT, radg + (size_t)J * kT, b_full + (J & 1));
+                ++loads[J & 1];
+            };
+            for (int J = 0; J <= I && J < 2; ++J) load_col(J);
             const uint32_t a_base = smem_u32(smem + OFF_A);
             bool ok = true;
             for (int J = 0; J <= I && ok; ++J) {
@@ -143,7 +165,7 @@ __global__ void __launch_bounds__(kThr, 1) k_pair_tc(const RbsArgs a, int nTB)
                 }
                 ok = ok && mbar_wait(b_full + s, (uint32_t)(J >> 1) & 1u, deadline, abort_flag);
                 if (ok) ++waited[s];
-                // the epilogue of column J - 2 has read accumulator s
+                // the epilogue of column J - 2 is done with accumulator s
                 if (ok && J >= 2) ok = mbar_wait(acc_free + s, (uint32_t)((J - 2) >> 1) & 1u, deadline, abort_flag);
                 if (!ok) break;
                 fence_after_sync();
@@ -163,8 +185,7 @@ __global__ void __launch_bounds__(kThr, 1) k_pair_tc(const RbsArgs a, int nTB)
                     const int o = s ^ 1;
                     ok = mbar_wait(mma_done + o, (uint32_t)((J - 1) >> 1) & 1u, deadline, abort_flag);
                     if (!ok) break;
-                    load_image(smem + OFF_B + o * kRbsImgBytes, cimg + (size_t)(J + 1) * kRbsImgBytes, b_full + o);
-                    ++loads[o];
+                    load_col(J + 1);
                 }
             }
             if (!ok) {
@@ -182,17 +203,16 @@ __global__ void __launch_bounds__(kThr, 1) k_pair_tc(const RbsArgs a, int nTB)
     } else {
         // ---------------- epilogue ----------------
         const int quarter = warp & 3, colh = warp >> 2;
-        const int i = I * kT + 32 * quarter + lane;   // this thread's query block
+        const int row0 = I * kT + 32 * quarter;
+        const int i = row0 + lane;   // this thread's query block
         const bool row_ok = i < a.nB;
         const float qn = row_ok ? a.qnorm[(size_t)h * a.nB + i] : 0.f;
-        const float tc = QUANT ? 0.f : __ldg(a.tau_c + h);
-        const float tr = QUANT ? 0.f : __ldg(a.tau_r + h);
+        const float tcs = QUANT ? 0.f : __ldg(a.tau_c + h) / a.scale;
+        const float trs = QUANT ? 0.f : __ldg(a.tau_r + h) / a.scale;
         const size_t nP = (size_t)a.nB * (a.nB + 1) / 2;
         const int words = rbs_mask_words(a.nB);
-        const float *radg = a.rad + (size_t)g * a.nB;
-        // 16-byte radius loads only where the kv head's row starts aligned
-        const bool rad16 = (reinterpret_cast<uintptr_t>(radg) & 15) == 0;
         const float2 sc2 = make_float2(a.scale, a.scale), qn2 = make_float2(qn, qn);
+        float *stg = reinterpret_cast<float *>(smem + OFF_STG) + warp * 32 * kStgStride;
         int kept = 0;
         for (int J = 0; J <= I; ++J) {
             const int s = J & 1;
@@ -210,62 +230,72 @@ __global__ void __launch_bounds__(kThr, 1) k_pair_tc(const RbsArgs a, int nTB)
             tmem_ld32(ta, v[0]);
             tmem_ld32(ta + 32, v[1]);
             tmem_wait_ld();
-            fence_before_sync();
-            mbar_arrive(acc_free + s);
+            const float *rs = srad + (J % kRadStages) * kT + 64 * colh;
             const int j0 = J * kT + 64 * colh;
-            // interior column tiles hold neither the diagonal nor block 0, and
-            // every pair in them is causal
-            const bool edge = J == 0 || J == I;
+            if constexpr (!QUANT) {
+                // S_c > tau_c  <=>  qc > tau_c / scale, and S_r > tau_r  <=>
+                // qc + qn r > tau_r / scale (scale > 0): one FMA, two
+                // compares and one predicated OR per pair
 #pragma unroll
-            for (int t = 0; t < 2; ++t) {
-                uint32_t word = 0;
+                for (int t = 0; t < 2; ++t) {
+                    uint32_t word = 0;
 #pragma unroll
-                for (int c8 = 0; c8 < 32; c8 += 8) {
-                    const int jb = j0 + 32 * t + c8;
-                    float rr[8];
-                    if (rad16 && jb + 8 <= a.nB) {
-                        const float4 r0 = __ldg(reinterpret_cast<const float4 *>(radg + jb));
-                        const float4 r1 = __ldg(reinterpret_cast<const float4 *>(radg + jb + 4));
-                        rr[0] = r0.x; rr[1] = r0.y; rr[2] = r0.z; rr[3] = r0.w;
-                        rr[4] = r1.x; rr[5] = r1.y; rr[6] = r1.z; rr[7] = r1.w;
-                    } else {
+                    for (int c = 0; c < 32; c += 4) {
+                        const float4 r4 = *reinterpret_cast<const float4 *>(rs + 32 * t + c);
+                        const float rr[4] = {r4.x, r4.y, r4.z, r4.w};
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) rr[e] = jb + e < a.nB ? __ldg(radg + jb + e) : 0.f;
+                        for (int e = 0; e < 4; ++e) {
+                            const float qc = __uint_as_float(v[t][c + e]);
+                            if (qc > tcs || fmaf(qn, rr[e], qc) > trs) word |= 1u << (c + e);
+                        }
+                    }
+                    const int jt = j0 + 32 * t;   // column of bit 0
+                    if (J == I) {
+                        // diagonal tile: causal bits only, diagonal forced
+                        const int dd = i - jt;     // bit of j == i
+                        word &= dd >= 31 ? 0xffffffffu : (dd < 0 ? 0u : (2u << dd) - 1u);
+                        if (a.force_diag && dd >= 0 && dd < 32) word |= 1u << dd;
+                    }
+                    if (a.force_first && jt == 0) word |= 1u;
+                    if (row_ok) {
+                        a.bits[((size_t)h * a.nB + i) * words + J * 4 + 2 * colh + t] = word;
+                        kept += __popc(word);
+                    }
+                }
+            } else {
+                // both scores of every causal pair, 16 columns at a time, staged
+                // through shared memory so that each store instruction writes
+                // two rows x 16 consecutive pairs
+#pragma unroll
+                for (int c16 = 0; c16 < 64; c16 += 16) {
+                    const int t = c16 >> 5, cb = c16 & 31;
+                    float sc[16], sr[16];
+#pragma unroll
+                    for (int e = 0; e < 16; e += 2) {
+                        const float2 q2 = make_float2(__uint_as_float(v[t][cb + e]), __uint_as_float(v[t][cb + e + 1]));
+                        const float2 x = fmul2(sc2, q2);
+                        const float2 y = fmul2(sc2, ffma2(qn2, make_float2(rs[c16 + e], rs[c16 + e + 1]), q2));
+                        sc[e] = x.x; sc[e + 1] = x.y; sr[e] = y.x; sr[e + 1] = y.y;
                     }
 #pragma unroll
-                    for (int e = 0; e < 8; e += 2) {
-                        const int c = c8 + e;
-                        const float2 qc = make_float2(__uint_as_float(v[t][c]), __uint_as_float(v[t][c + 1]));
-                        const float2 sc = fmul2(sc2, qc);
-                        const float2 sr = fmul2(sc2, ffma2(qn2, make_float2(rr[e], rr[e + 1]), qc));
-                        if (QUANT) {
-                            const int j = jb + e;
-                            if (row_ok && j <= i) {
-                                const size_t p = (size_t)i * (i + 1) / 2 + j;
-                                a.pair_sc[(size_t)h * nP + p] = sc.x;
-                                a.pair_sc[((size_t)a.Hq + h) * nP + p] = sr.x;
-                                if (j + 1 <= i) {
-                                    a.pair_sc[(size_t)h * nP + p + 1] = sc.y;
-                                    a.pair_sc[((size_t)a.Hq + h) * nP + p + 1] = sr.y;
-                                }
-                            }
-                        } else {
-                            bool k0 = sc.x > tc || sr.x > tr;
-                            bool k1 = sc.y > tc || sr.y > tr;
-                            if (edge) {
-                                const int j = jb + e;
-                                k0 = j <= i && (k0 || (a.force_diag && j == i) || (a.force_first && j == 0));
-                                k1 = j + 1 <= i && (k1 || (a.force_diag && j + 1 == i));
-                            }
-                            word |= ((uint32_t)k0 << c) | ((uint32_t)k1 << (c + 1));
+                    for (int br = 0; br < 2; ++br) {
+                        __syncwarp();
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) stg[lane * kStgStride + e] = br ? sr[e] : sc[e];
+                        __syncwarp();
+                        float *dst = a.pair_sc + ((size_t)br * a.Hq + h) * nP;
+                        const int col = lane & 15, j = j0 + c16 + col;
+#pragma unroll 4
+                        for (int r2 = 0; r2 < 32; r2 += 2) {
+                            const int rr = r2 + (lane >> 4), ir = row0 + rr;
+                            if (ir < a.nB && j <= ir) dst[(size_t)ir * (ir + 1) / 2 + j] = stg[rr * kStgStride + col];
                         }
                     }
                 }
-                if (!QUANT && row_ok) {
-                    a.bits[((size_t)h * a.nB + i) * words + J * 4 + 2 * colh + t] = word;
-                    kept += __popc(word);
-                }
             }
+            // this column's accumulator and radii stage are no longer read
+            fence_before_sync();
+            mbar_arrive(acc_free + s);
         }
         if (!QUANT && row_ok && kept) atomicAdd(&a.rowcnt[h * a.nB + i], kept);
     }

@@ -37,7 +37,7 @@ size_t rbs_workspace_layout(int Hq, int Hkv, int D, int nB, bool quantile, size_
     size_t o = 0;
     const size_t img = (size_t)rbs_img_tiles(nB) * kRbsImgBytes;   // per matrix (D = 128)
     offs[0] = o; o += up((size_t)Hkv * img);              // centroid tile images
-    offs[1] = o; o += up((size_t)Hkv * nB * 4);           // radii
+    offs[1] = o; o += up((size_t)Hkv * rbs_img_tiles(nB) * kRbsImgRows * 4);   // radii, rows padded to whole tiles
     offs[2] = o; o += up((size_t)Hq * img);               // pooled-query tile images
     offs[3] = o; o += up((size_t)Hq * nB * 4);            // pooled query norms
     offs[4] = o; o += up((size_t)2 * Hq * 4);             // thresholds
@@ -73,12 +73,14 @@ __global__ void __launch_bounds__(256) k_block_stats(const RbsArgs a)
     __shared__ float cen[D];
     __shared__ float wmax[8];
     const int j = blockIdx.x, g = blockIdx.y;
+    const int rad_rows = rbs_img_tiles(a.nB) * kRbsImgRows;
     uint8_t *img = a.cen + ((size_t)g * rbs_img_tiles(a.nB) + (j >> 7)) * kRbsImgBytes;
     if (j >= a.nB) {   // padding row of the last tile image
         if (threadIdx.x < D) {
             *reinterpret_cast<uint16_t *>(img + rbs_img_offset(j & 127, threadIdx.x, 0)) = 0;
             *reinterpret_cast<uint16_t *>(img + rbs_img_offset(j & 127, threadIdx.x, 1)) = 0;
         }
+        if (threadIdx.x == 0) a.rad[(size_t)g * rad_rows + j] = 0.f;
         return;
     }
     const int n = min(BS, a.T - j * BS);
@@ -124,7 +126,7 @@ __global__ void __launch_bounds__(256) k_block_stats(const RbsArgs a)
     if (threadIdx.x == 0) {
         float m = 0.f;
         for (int w = 0; w < 8; ++w) m = fmaxf(m, wmax[w]);
-        a.rad[(size_t)g * a.nB + j] = m;
+        a.rad[(size_t)g * rad_rows + j] = m;
     }
 }
 

@@ -316,7 +316,7 @@ sa_status sa_select_blocks(const sa_kv_cache *kv, const sa_block_select_args *ar
     if ((args->tau_c == nullptr) != (args->tau_r == nullptr)) return SA_ERR_INVALID_ARGUMENT;
     if (!args->tau_c && !(args->p_c >= 0.f && args->p_c <= 1.f && args->p_r >= 0.f && args->p_r <= 1.f))
         return SA_ERR_INVALID_ARGUMENT;
-    if (!(args->scale == args->scale)) return SA_ERR_INVALID_ARGUMENT;
+    if (!(args->scale > 0.f) || args->scale == INFINITY) return SA_ERR_INVALID_ARGUMENT;
     if (!out->row_ptr || !out->cols || out->nnz_capacity < 0) return SA_ERR_INVALID_ARGUMENT;
     const int nB = (T + bs - 1) / bs;
     if (nB > 65536) return SA_ERR_UNSUPPORTED;

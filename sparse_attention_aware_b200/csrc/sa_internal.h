@@ -97,7 +97,7 @@ struct RbsArgs {
     int force_diag, force_first;
     // workspace pieces
     uint8_t *cen;    // centroids, tile images [Hkv][nTB][64 KB] (rbs_img_offset)
-    float *rad;      // [Hkv][nB]
+    float *rad;      // [Hkv][nTB * 128] (rows past nB are 0)
     uint8_t *qbar;   // pooled queries, tile images [Hq][nTB][64 KB]
     float *qnorm;    // [Hq][nB]
     float *tau;      // [2][Hq] thresholds in use

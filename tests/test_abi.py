@@ -138,6 +138,11 @@ def test_host_validation_rejects_before_launch(lib):
     o.row_ptr, o.cols, o.nnz_capacity = 0x80000, 0x90000, 100
     assert lib.sa_select_blocks(ctypes.byref(kv64), ctypes.byref(a), ctypes.byref(o), 0x100000, 1 << 30,
                                 None) == INV             # quantile outside [0, 1]
+    a.p_c = 0.9
+    for bad_scale in (0.0, -0.1, float("inf"), float("nan")):
+        a.scale = bad_scale
+        assert lib.sa_select_blocks(ctypes.byref(kv64), ctypes.byref(a), ctypes.byref(o), 0x100000, 1 << 30,
+                                    None) == INV         # the selection scale must be finite and > 0
     a.mode = L.SEL_SPANS
     a.max_spans = 2000
     assert lib.sa_select_blocks(ctypes.byref(kv), ctypes.byref(a), ctypes.byref(o), 0x100000, 1 << 30,
