@@ -7,10 +7,10 @@
 //
 // B200 design.  tcgen05 MMAs run at full rate with M = 128 rows, while a
 // query block has 64.  One CTA therefore serves a work item of two 64-row
-// halves that share their K/V tiles: two query heads of one GQA group at the
-// same query block (the pairing is chosen per block by k_prefill_schedule,
-// greedily by the overlap of their CSR rows), or, for odd group sizes, two
-// adjacent query blocks of one head.  The CTA walks the union of the two rows;
+// halves that share their K/V tiles: two rows (query head, query block) of
+// one GQA group, from a window of nearby query blocks (the pairing is chosen
+// by k_prefill_schedule_window, greedily by the key blocks the two rows do not
+// share), or, for odd group sizes, two adjacent query blocks of one head.  The CTA walks the union of the two rows;
 // a key block listed by one half only is masked (p = 0) for the other half.
 //   warp 0      K producer: the Q halves (3-D map over [T][Hq][128]), then
 //               per key block of the merged list the K page tile (2-D map over
@@ -482,66 +482,117 @@ __global__ void __launch_bounds__(kThreads, 2)
 }
 
 // ---------------------------------------------------------------------------
-// Work items.  Even GQA group sizes (<= 16): per (kv head g, query block i),
-// pair the group's query heads greedily by the waste of their union (|A| +
-// |B| - 2|A n B|, smallest first, ties to the lowest pair).  One warp per
-// (g, i).  Items are ordered by kv head, then query block, latest first.
+// Work items.  Even GQA group sizes (<= 16): the rows (query head, query
+// block) of one kv head are paired within windows of Wq = 64 / G consecutive
+// query blocks, so a window holds G * Wq <= 64 rows of the group.  A pair's
+// waste is |A xor B|, the key blocks listed by one row only, which the CTA
+// executes for both halves; rows are paired greedily, smallest waste first,
+// ties to the lowest pair index.  Wastes come from per-row bitmaps in shared
+// memory (popcounts of xor), over chunks of kSchedBits key blocks.  One CTA
+// per (kv head, window); items are ordered kv-head-major, latest windows
+// first.
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_prefill_schedule_pairs(const PrefillArgs a)
+constexpr int kSchedRows = 64;
+constexpr int kSchedWords = 64;                 // bitmap words per row per chunk
+constexpr int kSchedBits = 32 * kSchedWords;    // key blocks per chunk
+constexpr int kSchedPairs = kSchedRows * (kSchedRows - 1) / 2;
+
+__device__ __forceinline__ int pair_index(int ka, int kb, int nc)
+{
+    return ka * nc - ka * (ka + 1) / 2 + (kb - ka - 1);
+}
+
+__global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillArgs a)
 {
     pdl_wait();
     pdl_trigger();
-    __shared__ int cost[8][kMaxPairGroup][kMaxPairGroup];
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    __shared__ uint32_t bits[kSchedRows][kSchedWords + 1];   // +1: conflict-free column reads
+    __shared__ int cost[kSchedPairs];
+    __shared__ int red_c[8], red_p[8];
+    __shared__ unsigned long long used;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nQB = (a.T + 63) >> 6;
     const int G = a.Hq / a.c.Hkv;
-    const int task = blockIdx.x * 8 + warp;
-    if (task >= a.c.Hkv * nQB) return;
-    const int g = task / nQB, i = task % nQB;
-    const int npairs = G * (G - 1) / 2;
-    for (int p = lane; p < npairs; p += 32) {
-        int x = 0, pa = 0, pb = 1;
-        for (pa = 0; pa < G - 1; ++pa) {
-            if (p < x + (G - 1 - pa)) {
-                pb = pa + 1 + (p - x);
-                break;
+    const int Wq = kSchedRows / G;
+    const int nW = (nQB + Wq - 1) / Wq;
+    const int g = blockIdx.x / nW, I = blockIdx.x % nW;
+    if (g >= a.c.Hkv) return;
+    const int i0 = I * Wq, i1 = min(i0 + Wq, nQB);
+    const int nc = G * (i1 - i0);                // even: G is even
+    const int np = nc * (nc - 1) / 2;
+    // row k of the window: head g*G + k % G, query block i0 + k / G
+    for (int p = tid; p < np; p += 256) cost[p] = 0;
+    for (int kb0 = 0; kb0 < i1; kb0 += kSchedBits) {
+        __syncthreads();
+        for (int w = tid; w < nc * kSchedWords; w += 256) bits[w / kSchedWords][w % kSchedWords] = 0u;
+        __syncthreads();
+        for (int k = warp; k < nc; k += 8) {
+            const int i = i0 + k / G;
+            const int32_t *c;
+            const int n = csr_row(a, (g * G + k % G) * nQB + i, i, c);
+            for (int e = lane; e < n; e += 32) {
+                const int rel = __ldg(c + e) - kb0;   // out-of-range entries are the kernel's to record
+                if (rel >= 0 && rel < kSchedBits && rel + kb0 <= i) atomicOr(&bits[k][rel >> 5], 1u << (rel & 31));
             }
-            x += G - 1 - pa;
         }
-        const int32_t *ca, *cb;
-        const int na = csr_row(a, (g * G + pa) * nQB + i, i, ca);
-        const int nb = csr_row(a, (g * G + pb) * nQB + i, i, cb);
-        int ia = 0, ib = 0, inter = 0;
-        while (ia < na && ib < nb) {
-            const int va = __ldg(ca + ia), vb = __ldg(cb + ib);
-            inter += va == vb;
-            ia += va <= vb;
-            ib += vb <= va;
+        __syncthreads();
+        const int words = min(kSchedWords, (i1 - kb0 + 31) >> 5);
+        for (int ka = warp; ka < nc; ka += 8) {
+            for (int kb = ka + 1 + lane; kb < nc; kb += 32) {
+                int x = 0;
+                for (int w = 0; w < words; ++w) x += __popc(bits[ka][w] ^ bits[kb][w]);
+                cost[pair_index(ka, kb, nc)] += x;
+            }
         }
-        cost[warp][pa][pb] = na + nb - 2 * inter;
     }
-    __syncwarp();
-    if (lane == 0) {
-        unsigned used = 0;
-        // kv-head-major: CTAs in flight share one kv head's K/V (64 MB at 128K
-        // tokens), which then stays in L2; within a head, latest blocks first
-        const int base = g * nQB * (G / 2) + (nQB - 1 - i) * (G / 2);
-        for (int t = 0; t < G / 2; ++t) {
-            int best = INT_MAX, ba = 0, bb = 1;
-            for (int pa = 0; pa < G; ++pa) {
-                if (used >> pa & 1) continue;
-                for (int pb = pa + 1; pb < G; ++pb) {
-                    if (used >> pb & 1) continue;
-                    if (cost[warp][pa][pb] < best) {
-                        best = cost[warp][pa][pb];
-                        ba = pa;
-                        bb = pb;
-                    }
+    if (tid == 0) used = 0ull;
+    __syncthreads();
+    const int base = g * nQB * (G / 2) + (nQB - i1) * (G / 2);
+    for (int t = 0; t < nc / 2; ++t) {
+        const unsigned long long u = used;
+        int bc = INT_MAX, bp = INT_MAX;
+        for (int ka = warp; ka < nc; ka += 8) {
+            if (u >> ka & 1ull) continue;
+            for (int kb = ka + 1 + lane; kb < nc; kb += 32) {
+                if (u >> kb & 1ull) continue;
+                const int p = pair_index(ka, kb, nc), c = cost[p];
+                if (c < bc || (c == bc && p < bp)) {
+                    bc = c;
+                    bp = p;
                 }
             }
-            used |= (1u << ba) | (1u << bb);
-            a.items[base + t] = make_int4(g * G + ba, i, g * G + bb, i);
         }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const int oc = __shfl_xor_sync(0xffffffffu, bc, o), op = __shfl_xor_sync(0xffffffffu, bp, o);
+            if (oc < bc || (oc == bc && op < bp)) {
+                bc = oc;
+                bp = op;
+            }
+        }
+        if (lane == 0) {
+            red_c[warp] = bc;
+            red_p[warp] = bp;
+        }
+        __syncthreads();
+        if (tid == 0) {
+            for (int w = 1; w < 8; ++w)
+                if (red_c[w] < bc || (red_c[w] == bc && red_p[w] < bp)) {
+                    bc = red_c[w];
+                    bp = red_p[w];
+                }
+            if (bp >= np) bp = 0;   // unreachable: an even count of unpaired rows remains
+            // decode the pair index
+            int ka = 0, rem = bp;
+            while (rem >= nc - 1 - ka) {
+                rem -= nc - 1 - ka;
+                ++ka;
+            }
+            const int kb = ka + 1 + rem;
+            used = u | (1ull << ka) | (1ull << kb);
+            a.items[base + t] = make_int4(g * G + ka % G, i0 + ka / G, g * G + kb % G, i0 + kb / G);
+        }
+        __syncthreads();
     }
 }
 
@@ -602,7 +653,8 @@ cudaError_t launch_prefill(const PrefillArgs &a, cudaStream_t s)
     const int G = a.Hq / a.c.Hkv;
     if (a.n_items <= 0) return cudaSuccess;
     if (G % 2 == 0 && G <= kMaxPairGroup) {
-        if (cudaError_t e_ = launch_pdl(k_prefill_schedule_pairs, dim3((a.c.Hkv * nQB + 7) / 8), dim3(256), 0, s, a))
+        const int nW = (nQB + kSchedRows / G - 1) / (kSchedRows / G);
+        if (cudaError_t e_ = launch_pdl(k_prefill_schedule_window, dim3(a.c.Hkv * nW), dim3(256), 0, s, a))
             return e_;
     } else {
         if (cudaError_t e_ = launch_pdl(k_prefill_schedule_adjacent, dim3((a.n_items + 255) / 256), dim3(256), 0, s, a))
