@@ -240,7 +240,9 @@ SA_API sa_status sa_select_blocks(const sa_kv_cache *kv, const sa_block_select_a
  * empty set gives out = 0 and lse = -inf.
  * Block lists (one list per sequence, shared by every head) with at most 16
  * query heads per kv head are computed per GQA group on tensor cores: the
- * parts are runs of list entries balanced by entry count, S = q.k is
+ * parts are runs of list entries balanced by entry count, a sequence using
+ * only as many of the num_splits parts as give each at least ~128 tokens
+ * (max(1, 128 / page_size) entries; the rest stay empty), S = q.k is
  * accumulated in fp32 (an fp32 query as bf16 high + low parts), and the
  * softmax weights enter the P.V product as bf16.
  *   q        [batch][num_q_heads][head_dim], fp32 or bf16

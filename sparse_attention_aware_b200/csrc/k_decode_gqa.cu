@@ -14,7 +14,8 @@
 //
 // One CTA = (split s, kv head g, sequence b), 4 warps.  The split owns a
 // contiguous range of the sequence's list entries (balanced by entry count;
-// an entry is at most one page).  Entries are staged in shared memory in
+// an entry is at most one page); a sequence uses only as many of the S splits
+// as give each at least ~128 tokens.  Entries are staged in shared memory in
 // windows of up to kWin, validated, mapped to physical pages once, and
 // prefix-summed into positions; each entry's K and V rows are prefetched into
 // L2 right away (one bulk prefetch each), so the latency of the scattered page
@@ -35,6 +36,7 @@ constexpr int kGT = 64;                  // tokens per tile
 constexpr int kGWarps = 4;               // a warp owns 16 tokens of a tile
 constexpr int kGThreads = kGWarps * 32;
 constexpr int kWin = 512;                // list entries staged per window
+constexpr int kSplitTokens = 128;        // a split of a sequence's list covers at least ~this many tokens
 
 template <int D>
 struct GqaSmem {
@@ -146,7 +148,21 @@ __global__ void __launch_bounds__(kGThreads) k_decode_gqa_blocks(const DecodeArg
         if (tid == 0 && s == 0 && g == 0) fault(st, CHK_BLOCK_ENTRY, ne);
         ne = ne < 0 ? 0 : a.max_blocks;
     }
-    const int e0 = (int)((long long)ne * s / a.S), e1 = (int)((long long)ne * (s + 1) / a.S);
+    // The sequence uses Sb <= S splits of at least kSplitTokens / P entries
+    // each (an entry is at most one page), so a short list is not spread over
+    // many CTAs that each pay the fixed cost of a split; the splits past Sb
+    // leave an empty partial (l = 0), which the combine skips.
+    const int per = max(1, kSplitTokens >> a.c.Plog2);
+    const int Sb = min(a.S, max(1, (ne + per - 1) / per));
+    if (s >= Sb) {
+        for (int j = tid; j < min(HPG, 16); j += kGThreads) {
+            const size_t row = (size_t)b * a.Hq + g * HPG + j;
+            a.part_ml[(row * a.S + s) * 2 + 0] = -INFINITY;
+            a.part_ml[(row * a.S + s) * 2 + 1] = 0.f;
+        }
+        return;
+    }
+    const int e0 = (int)((long long)ne * s / Sb), e1 = (int)((long long)ne * (s + 1) / Sb);
     const int4 *ent = reinterpret_cast<const int4 *>(a.ent) + (size_t)b * a.max_blocks;
     const int32_t *ptb = a.c.pt + (size_t)b * a.c.max_pages;
     const int P = 1 << a.c.Plog2;
