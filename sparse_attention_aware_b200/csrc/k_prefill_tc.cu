@@ -487,7 +487,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 // query blocks, so a window holds G * Wq <= 64 rows of the group.  A pair's
 // waste is |A xor B|, the key blocks listed by one row only, which the CTA
 // executes for both halves; rows are paired greedily, smallest waste first,
-// ties to the lowest pair index.  Wastes come from per-row bitmaps in shared
+// ties to the lowest pair index, then improved by 2-opt exchanges.  Wastes come from per-row bitmaps in shared
 // memory (popcounts of xor), over chunks of kSchedBits key blocks.  One CTA
 // per (kv head, window); items are ordered kv-head-major, latest windows
 // first.
@@ -509,6 +509,7 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
     __shared__ uint32_t bits[kSchedRows][kSchedWords + 1];   // +1: conflict-free column reads
     __shared__ int cost[kSchedPairs];
     __shared__ int red_c[8], red_p[8];
+    __shared__ int pr_a[kSchedRows / 2], pr_b[kSchedRows / 2];
     __shared__ unsigned long long used;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nQB = (a.T + 63) >> 6;
@@ -590,9 +591,78 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
             }
             const int kb = ka + 1 + rem;
             used = u | (1ull << ka) | (1ull << kb);
-            a.items[base + t] = make_int4(g * G + ka % G, i0 + ka / G, g * G + kb % G, i0 + kb / G);
+            pr_a[t] = ka;
+            pr_b[t] = kb;
         }
         __syncthreads();
+    }
+    // 2-opt: repeatedly apply the exchange of partners between two pairs that
+    // lowers the total waste most (ties to the lowest pair of pairs), until
+    // none does
+    const int npr = nc / 2, nsw = npr * (npr - 1) / 2;
+    auto cst = [&](int x, int y) { return cost[x < y ? pair_index(x, y, nc) : pair_index(y, x, nc)]; };
+    for (int it = 0; it < 4 * kSchedRows; ++it) {
+        int bg = 0, bq = INT_MAX;   // best gain (> 0), its exchange index and kind (bit 0)
+        for (int q = tid; q < nsw; q += 256) {
+            int x = 0, rem = q;
+            while (rem >= npr - 1 - x) {
+                rem -= npr - 1 - x;
+                ++x;
+            }
+            const int y = x + 1 + rem;
+            const int ax = pr_a[x], bx = pr_b[x], ay = pr_a[y], by = pr_b[y];
+            const int cur = cst(ax, bx) + cst(ay, by);
+            const int o1 = cst(ax, ay) + cst(bx, by), o2 = cst(ax, by) + cst(bx, ay);
+            const int gain = cur - min(o1, o2);
+            const int code = 2 * q + (o1 <= o2 ? 0 : 1);
+            if (gain > bg || (gain == bg && gain > 0 && code < bq)) {
+                bg = gain;
+                bq = code;
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            const int og = __shfl_xor_sync(0xffffffffu, bg, o), oq = __shfl_xor_sync(0xffffffffu, bq, o);
+            if (og > bg || (og == bg && oq < bq)) {
+                bg = og;
+                bq = oq;
+            }
+        }
+        if (lane == 0) {
+            red_c[warp] = bg;
+            red_p[warp] = bq;
+        }
+        __syncthreads();
+        bg = red_c[0];
+        bq = red_p[0];
+        for (int w = 1; w < 8; ++w)
+            if (red_c[w] > bg || (red_c[w] == bg && red_p[w] < bq)) {
+                bg = red_c[w];
+                bq = red_p[w];
+            }
+        __syncthreads();                 // every thread has read red_*
+        if (bg <= 0) break;              // uniform: every thread reduced the same values
+        if (tid == 0) {
+            int x = 0, rem = bq >> 1;
+            while (rem >= npr - 1 - x) {
+                rem -= npr - 1 - x;
+                ++x;
+            }
+            const int y = x + 1 + rem;
+            const int bx = pr_b[x];
+            if ((bq & 1) == 0) {         // (ax, ay), (bx, by)
+                pr_b[x] = pr_a[y];
+                pr_a[y] = bx;
+            } else {                     // (ax, by), (bx, ay)
+                pr_b[x] = pr_b[y];
+                pr_b[y] = bx;
+            }
+        }
+        __syncthreads();
+    }
+    for (int t = tid; t < npr; t += 256) {
+        const int ka = pr_a[t], kb = pr_b[t];
+        a.items[base + t] = make_int4(g * G + ka % G, i0 + ka / G, g * G + kb % G, i0 + kb / G);
     }
 }
 
