@@ -510,7 +510,6 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
     __shared__ int cost[kSchedPairs];
     __shared__ int red_c[8], red_p[8];
     __shared__ int pr_a[kSchedRows / 2], pr_b[kSchedRows / 2];
-    __shared__ unsigned long long used;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nQB = (a.T + 63) >> 6;
     const int G = a.Hq / a.c.Hkv;
@@ -546,56 +545,65 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
             }
         }
     }
-    if (tid == 0) used = 0ull;
+    // greedy pairing = one pass over the pairs in ascending (waste, row a,
+    // row b) order, taking a pair when both rows are still free.  Keys
+    // (waste clamped to 20 bits, then the two 6-bit row ids) are bitonic-sorted
+    // in the bitmap's shared memory, which is free now.
+    uint32_t *keys = &bits[0][0];
+    constexpr int kKeys = 2048;   // >= kSchedPairs, power of two
+    static_assert(kKeys >= kSchedPairs && kKeys <= kSchedRows * (kSchedWords + 1), "key buffer");
+    __syncthreads();
+    for (int ka = warp; ka < kSchedRows; ka += 8) {
+        for (int kb = ka + 1 + lane; kb < kSchedRows; kb += 32) {
+            const int p = pair_index(ka, kb, kSchedRows);
+            uint32_t key = 0xFFFFFFFFu;
+            if (kb < nc) key = ((uint32_t)min(cost[pair_index(ka, kb, nc)], (1 << 20) - 1) << 12) | (ka << 6) | kb;
+            keys[p] = key;
+        }
+    }
+    for (int p = kSchedPairs + tid; p < kKeys; p += 256) keys[p] = 0xFFFFFFFFu;
+    for (int kk = 2; kk <= kKeys; kk <<= 1) {
+        for (int j = kk >> 1; j > 0; j >>= 1) {
+            __syncthreads();
+            for (int i = tid; i < kKeys; i += 256) {
+                const int ixj = i ^ j;
+                if (ixj > i) {
+                    const uint32_t x = keys[i], y = keys[ixj];
+                    const bool up = (i & kk) == 0;
+                    if ((x > y) == up) {
+                        keys[i] = y;
+                        keys[ixj] = x;
+                    }
+                }
+            }
+        }
+    }
     __syncthreads();
     const int base = g * nQB * (G / 2) + (nQB - i1) * (G / 2);
-    for (int t = 0; t < nc / 2; ++t) {
-        const unsigned long long u = used;
-        int bc = INT_MAX, bp = INT_MAX;
-        for (int ka = warp; ka < nc; ka += 8) {
-            if (u >> ka & 1ull) continue;
-            for (int kb = ka + 1 + lane; kb < nc; kb += 32) {
-                if (u >> kb & 1ull) continue;
-                const int p = pair_index(ka, kb, nc), c = cost[p];
-                if (c < bc || (c == bc && p < bp)) {
-                    bc = c;
-                    bp = p;
+    if (warp == 0) {
+        unsigned long long u = 0ull;
+        int t = 0;
+        for (int q0 = 0; q0 < np && t < nc / 2; q0 += 32) {
+            const uint32_t key = keys[q0 + lane];   // q0 + lane < kKeys; padding keys sort last
+            const int ka = (key >> 6) & 63, kb = key & 63;
+            const bool cand = q0 + lane < np && !(u >> ka & 1ull) && !(u >> kb & 1ull);
+            unsigned m = __ballot_sync(0xffffffffu, cand);
+            while (m) {
+                const int l = __ffs(m) - 1;
+                m &= m - 1;
+                const int xa = __shfl_sync(0xffffffffu, ka, l), xb = __shfl_sync(0xffffffffu, kb, l);
+                if (!(u >> xa & 1ull) && !(u >> xb & 1ull)) {
+                    u |= (1ull << xa) | (1ull << xb);
+                    if (lane == 0) {
+                        pr_a[t] = xa;
+                        pr_b[t] = xb;
+                    }
+                    ++t;
                 }
             }
         }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            const int oc = __shfl_xor_sync(0xffffffffu, bc, o), op = __shfl_xor_sync(0xffffffffu, bp, o);
-            if (oc < bc || (oc == bc && op < bp)) {
-                bc = oc;
-                bp = op;
-            }
-        }
-        if (lane == 0) {
-            red_c[warp] = bc;
-            red_p[warp] = bp;
-        }
-        __syncthreads();
-        if (tid == 0) {
-            for (int w = 1; w < 8; ++w)
-                if (red_c[w] < bc || (red_c[w] == bc && red_p[w] < bp)) {
-                    bc = red_c[w];
-                    bp = red_p[w];
-                }
-            if (bp >= np) bp = 0;   // unreachable: an even count of unpaired rows remains
-            // decode the pair index
-            int ka = 0, rem = bp;
-            while (rem >= nc - 1 - ka) {
-                rem -= nc - 1 - ka;
-                ++ka;
-            }
-            const int kb = ka + 1 + rem;
-            used = u | (1ull << ka) | (1ull << kb);
-            pr_a[t] = ka;
-            pr_b[t] = kb;
-        }
-        __syncthreads();
     }
+    __syncthreads();
     // 2-opt: repeatedly apply the exchange of partners between two pairs that
     // lowers the total waste most (ties to the lowest pair of pairs), until
     // none does
