@@ -45,10 +45,10 @@ TILE_FLOPS = 4 * 64 * 64 * 128
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 # kernels each API call launches (libsa): top-k = score + select; decode =
-# split + combine; spans = 1; RBS with explicit thresholds = stats, pooling,
-# threshold copy, pair tiles, 3 CSR scan kernels, CSR fill, threshold copy-out;
-# prefill = schedule + tcgen05 kernel
-LAUNCHES = {"select_topk": 2, "decode": 2, "spans": 1, "rbs_explicit": 9, "prefill": 2}
+# split + combine; spans = 1; RBS with explicit thresholds = block statistics,
+# query pooling, pair tiles, 3 CSR scan kernels, CSR fill; prefill = schedule +
+# tcgen05 kernel
+LAUNCHES = {"select_topk": 2, "decode": 2, "spans": 1, "rbs_explicit": 7, "prefill": 2}
 
 
 def peaks():

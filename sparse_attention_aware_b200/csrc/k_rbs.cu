@@ -64,15 +64,28 @@ __device__ __forceinline__ void store_split(uint8_t *img, int row, int k, float 
 }
 
 // ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_block_stats(const RbsArgs a)
+// Block statistics (one CTA per key block and kv head) and query pooling (one
+// CTA per query block and q head), two launches over nB rounded up to whole
+// 128-row tile images, whose padding rows are zeroed.  The pooling CTA of
+// (i, h) also clears row i's mask count of head h, and the first statistics
+// CTA copies explicit thresholds into place.  (One launch with both kinds of
+// CTA was measured 10% slower.)
+// ---------------------------------------------------------------------------
+struct StatsSmem {
+    uint16_t tile[BS * 128];   // key block, bf16 rows
+    float cen[128];
+    float csum[2][128];
+    float wmax[8];
+    int page[BS];              // physical page of each page of the block (<= 64 pages)
+};
+struct PoolSmem {
+    float part[16][128];
+    float red[4];
+};
+
+__device__ void block_stats_cta(const RbsArgs &a, StatsSmem &sm, int j, int g)
 {
-    pdl_wait();
-    pdl_trigger();
     constexpr int D = 128;
-    __shared__ __align__(16) uint16_t tile[BS * D];
-    __shared__ float cen[D];
-    __shared__ float wmax[8];
-    const int j = blockIdx.x, g = blockIdx.y;
     const int rad_rows = rbs_img_tiles(a.nB) * kRbsImgRows;
     uint8_t *img = a.cen + ((size_t)g * rbs_img_tiles(a.nB) + (j >> 7)) * kRbsImgBytes;
     if (j >= a.nB) {   // padding row of the last tile image
@@ -85,26 +98,51 @@ __global__ void __launch_bounds__(256) k_block_stats(const RbsArgs a)
     }
     const int n = min(BS, a.T - j * BS);
     const int P = 1 << a.c.Plog2;
-    // stage the block's rows (16-byte chunks; 16 per row)
-    for (int ch = threadIdx.x; ch < n * (D / 8); ch += blockDim.x) {
-        const int r = ch >> 4, c8 = ch & 15;
-        const int t = j * BS + r;
-        int page = __ldg(a.c.pt + (t >> a.c.Plog2));
-        uint4 v = make_uint4(0, 0, 0, 0);
+    // pages of the block (one at P = 64): looked up once, not per row
+    const int npg = (n + P - 1) >> a.c.Plog2;
+    if (threadIdx.x < npg) {
+        int page = __ldg(a.c.pt + ((j * BS) >> a.c.Plog2) + threadIdx.x);
         if (page < 0 || page >= a.c.num_pages) {
             fault(a.st, CHK_PAGE, page);
-        } else {
-            const size_t off = ((((size_t)page * a.c.Hkv + g) << a.c.Plog2) + (t & (P - 1))) * D + c8 * 8;
-            v = ldg_nc_v4(a.c.k + off);
+            page = -1;
         }
-        *reinterpret_cast<uint4 *>(&tile[r * D + c8 * 8]) = v;
+        sm.page[threadIdx.x] = page;
+    }
+    __syncthreads();
+    // stage the block's rows: 16-byte chunks, all of a thread's loads in flight at once
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int ch = threadIdx.x + u * 256;   // 64 rows x 16 chunks = 1024
+        const int r = ch >> 4, c8 = ch & 15;
+        v[u] = make_uint4(0, 0, 0, 0);
+        if (r < n) {
+            const int page = sm.page[r >> a.c.Plog2];
+            if (page >= 0) {
+                const size_t off = ((((size_t)page * a.c.Hkv + g) << a.c.Plog2) + (r & (P - 1))) * D + c8 * 8;
+                v[u] = ldg_nc_v4(a.c.k + off);
+            }
+        }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const int ch = threadIdx.x + u * 256;
+        *reinterpret_cast<uint4 *>(&sm.tile[(ch >> 4) * D + (ch & 15) * 8]) = v[u];
+    }
+    __syncthreads();
+    {   // column sums: two threads per column, rows interleaved, 4 chains each
+        const int col = threadIdx.x & (D - 1), half = threadIdx.x >> 7;
+        float s4[4] = {0.f, 0.f, 0.f, 0.f};
+        for (int r = half; r < n; r += 8)
+#pragma unroll
+            for (int q = 0; q < 4; ++q)
+                if (r + 2 * q < n) s4[q] += __uint_as_float((uint32_t)sm.tile[(r + 2 * q) * D + col] << 16);
+        sm.csum[half][col] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
     }
     __syncthreads();
     if (threadIdx.x < D) {
-        float s = 0.f;
-        for (int r = 0; r < n; ++r) s += __uint_as_float((uint32_t)tile[r * D + threadIdx.x] << 16);
-        const float c = s / (float)n;
-        cen[threadIdx.x] = c;
+        const float c = (sm.csum[0][threadIdx.x] + sm.csum[1][threadIdx.x]) / (float)n;
+        sm.cen[threadIdx.x] = c;
         store_split(img, j & 127, threadIdx.x, c);
     }
     __syncthreads();
@@ -115,30 +153,24 @@ __global__ void __launch_bounds__(256) k_block_stats(const RbsArgs a)
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
             const int col = lane * 4 + q;
-            const float dlt = __uint_as_float((uint32_t)tile[r * D + col] << 16) - cen[col];
+            const float dlt = __uint_as_float((uint32_t)sm.tile[r * D + col] << 16) - sm.cen[col];
             e = fmaf(dlt, dlt, e);
         }
         e = warp_sum(e);
         mx = fmaxf(mx, sqrtf(e));
     }
-    if (lane == 0) wmax[warp] = mx;
+    if (lane == 0) sm.wmax[warp] = mx;
     __syncthreads();
     if (threadIdx.x == 0) {
         float m = 0.f;
-        for (int w = 0; w < 8; ++w) m = fmaxf(m, wmax[w]);
+        for (int w = 0; w < 8; ++w) m = fmaxf(m, sm.wmax[w]);
         a.rad[(size_t)g * rad_rows + j] = m;
     }
 }
 
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_pool_q(const RbsArgs a)
+__device__ void pool_q_cta(const RbsArgs &a, PoolSmem &sm, int i, int h)
 {
-    pdl_wait();
-    pdl_trigger();
     constexpr int D = 128;
-    __shared__ float part[16][D];
-    __shared__ float red[4];
-    const int i = blockIdx.x, h = blockIdx.y;
     uint8_t *img = a.qbar + ((size_t)h * rbs_img_tiles(a.nB) + (i >> 7)) * kRbsImgBytes;
     if (i >= a.nB) {   // padding row of the last tile image
         if (threadIdx.x < D) {
@@ -147,6 +179,7 @@ __global__ void __launch_bounds__(256) k_pool_q(const RbsArgs a)
         }
         return;
     }
+    if (threadIdx.x == 0) a.rowcnt[(size_t)h * a.nB + i] = 0;
     const int n = min(BS, a.T - i * BS);
     const int lane16 = threadIdx.x & 15, rs = threadIdx.x >> 4;   // 16 row slots
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -157,21 +190,43 @@ __global__ void __launch_bounds__(256) k_pool_q(const RbsArgs a)
         acc[4] += bf_lo(w.z); acc[5] += bf_hi(w.z); acc[6] += bf_lo(w.w); acc[7] += bf_hi(w.w);
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e) part[rs][lane16 * 8 + e] = acc[e];
+    for (int e = 0; e < 8; ++e) sm.part[rs][lane16 * 8 + e] = acc[e];
     __syncthreads();
     float sq = 0.f;
     if (threadIdx.x < D) {
         float s = 0.f;
 #pragma unroll
-        for (int r = 0; r < 16; ++r) s += part[r][threadIdx.x];
+        for (int r = 0; r < 16; ++r) s += sm.part[r][threadIdx.x];
         const float qb = s / (float)n;
         store_split(img, i & 127, threadIdx.x, qb);
         sq = qb * qb;
     }
     sq = warp_sum(sq);
-    if ((threadIdx.x & 31) == 0 && threadIdx.x < D) red[threadIdx.x >> 5] = sq;
+    if ((threadIdx.x & 31) == 0 && threadIdx.x < D) sm.red[threadIdx.x >> 5] = sq;
     __syncthreads();
-    if (threadIdx.x == 0) a.qnorm[(size_t)h * a.nB + i] = sqrtf((red[0] + red[1]) + (red[2] + red[3]));
+    if (threadIdx.x == 0) a.qnorm[(size_t)h * a.nB + i] = sqrtf((sm.red[0] + sm.red[1]) + (sm.red[2] + sm.red[3]));
+}
+
+__global__ void __launch_bounds__(256) k_block_stats(const RbsArgs a)
+{
+    pdl_wait();
+    pdl_trigger();
+    __shared__ __align__(16) uint8_t raw[sizeof(StatsSmem)];
+    if (blockIdx.x == 0 && blockIdx.y == 0 && a.tau_c) {   // explicit thresholds
+        for (int h = threadIdx.x; h < a.Hq; h += blockDim.x) {
+            a.tau[h] = a.tau_c[h];
+            a.tau[a.Hq + h] = a.tau_r[h];
+        }
+    }
+    block_stats_cta(a, *reinterpret_cast<StatsSmem *>(raw), blockIdx.x, blockIdx.y);
+}
+
+__global__ void __launch_bounds__(256) k_pool_q(const RbsArgs a)
+{
+    pdl_wait();
+    pdl_trigger();
+    __shared__ __align__(16) uint8_t raw[sizeof(PoolSmem)];
+    pool_q_cta(a, *reinterpret_cast<PoolSmem *>(raw), blockIdx.x, blockIdx.y);
 }
 
 // ---------------------------------------------------------------------------
@@ -401,6 +456,8 @@ __global__ void __launch_bounds__(256) k_csr_fill(const RbsArgs a)
 {
     pdl_wait();
     pdl_trigger();
+    if (blockIdx.x == 0 && a.tau_out)
+        for (int x = threadIdx.x; x < 2 * a.Hq; x += blockDim.x) a.tau_out[x] = a.tau[x];
     const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= a.Hq * a.nB) return;
@@ -431,24 +488,6 @@ __global__ void __launch_bounds__(256) k_csr_fill(const RbsArgs a)
     }
 }
 
-__global__ void k_copy_tau(const RbsArgs a)
-{
-    pdl_wait();
-    pdl_trigger();
-    const int h = threadIdx.x + blockIdx.x * blockDim.x;
-    if (h >= a.Hq) return;
-    a.tau[h] = a.tau_c[h];
-    a.tau[a.Hq + h] = a.tau_r[h];
-}
-
-__global__ void k_tau_out(const RbsArgs a)
-{
-    pdl_wait();
-    pdl_trigger();
-    const int x = threadIdx.x + blockIdx.x * blockDim.x;
-    if (x < 2 * a.Hq) a.tau_out[x] = a.tau[x];
-}
-
 }  // namespace
 
 cudaError_t launch_rbs(const RbsArgs &a, cudaStream_t s)
@@ -458,8 +497,8 @@ cudaError_t launch_rbs(const RbsArgs &a, cudaStream_t s)
     cudaError_t e;
     // per-kv-head block statistics on sequence 0's keys
     const int img_rows = rbs_img_tiles(a.nB) * kRbsImgRows;   // padding rows are zeroed
-    if (cudaError_t e_ = launch_pdl(k_block_stats, dim3(dim3(img_rows, a.c.Hkv)), dim3(256), 0, s, a)) return e_;
-    if (cudaError_t e_ = launch_pdl(k_pool_q, dim3(dim3(img_rows, a.Hq)), dim3(256), 0, s, a)) return e_;
+    if (cudaError_t e_ = launch_pdl(k_block_stats, dim3(img_rows, a.c.Hkv), dim3(256), 0, s, a)) return e_;
+    if (cudaError_t e_ = launch_pdl(k_pool_q, dim3(img_rows, a.Hq), dim3(256), 0, s, a)) return e_;
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     if (quant) {
         if ((e = launch_pair_tc(a, true, s)) != cudaSuccess) return e;
@@ -472,8 +511,6 @@ cudaError_t launch_rbs(const RbsArgs &a, cudaStream_t s)
         }
         if (cudaError_t e_ = launch_pdl(k_mask_scores, dim3((a.Hq * a.nB + 7) / 8), dim3(256), 0, s, a)) return e_;
     } else {
-        if (cudaError_t e_ = launch_pdl(k_copy_tau, dim3((a.Hq + 127) / 128), dim3(128), 0, s, a)) return e_;
-        if ((e = cudaMemsetAsync(a.rowcnt, 0, (size_t)a.Hq * a.nB * sizeof(int32_t), s)) != cudaSuccess) return e;
         if ((e = launch_pair_tc(a, false, s)) != cudaSuccess) return e;
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -486,9 +523,6 @@ cudaError_t launch_rbs(const RbsArgs &a, cudaStream_t s)
         if (cudaError_t e_ = launch_pdl(k_csr_scan, dim3(nch), dim3(kScanChunk), 0, s, a, chunk)) return e_;
     }
     if (cudaError_t e_ = launch_pdl(k_csr_fill, dim3((a.Hq * a.nB + 7) / 8), dim3(256), 0, s, a)) return e_;
-    if (a.tau_out) {
-        if (cudaError_t e_ = launch_pdl(k_tau_out, dim3((2 * a.Hq + 127) / 128), dim3(128), 0, s, a)) return e_;
-    }
     return cudaGetLastError();
 }
 
