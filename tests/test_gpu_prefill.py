@@ -165,3 +165,46 @@ def test_bench_prefill_config(cuda_dev):
     g_out = out.float().cpu().numpy().reshape(-1, d)[rows]
     assert_close_attn(g_out, ref)
     np.testing.assert_allclose(lse.cpu().numpy().reshape(-1)[rows], ref_lse, atol=2e-3, rtol=0)
+
+
+def _schedule_items(ws, Hq, Hkv, nB):
+    """Work items the last prefill call left in its workspace (after the
+    256-byte status header): {head A, block A, head B (-1: none), block B}."""
+    G = Hq // Hkv
+    n_items = (Hq // 2) * nB if (G % 2 == 0 and G <= 16) else Hq * ((nB + 1) // 2)
+    buf = ws.buf
+    off = (-buf.data_ptr()) % 256 + 256
+    return buf[off: off + 16 * n_items].view(torch.int32).reshape(-1, 4).cpu().numpy()
+
+
+@pytest.mark.parametrize("T,Hq,Hkv", [(1500, 12, 2), (1500, 16, 1), (777, 6, 2), (1300, 2, 1), (2100, 8, 1)])
+def test_prefill_group_sizes_and_schedule(cuda_dev, T, Hq, Hkv):
+    """Group sizes 6 and 16 (rows paired within windows of 10 and 4 query
+    blocks, the last window partial), 2 and 8, and an odd group (adjacent
+    query blocks of one head); random masks with empty rows.  The work items
+    must cover every (head, query block) row exactly once, and the two halves
+    of an item must share a kv head."""
+    wl = W.random_prefill(700 + T + Hq, T, Hq, Hkv, 128, 64)
+    nB = (T + 63) // 64
+    mask = _random_mask(T + Hq, Hq, nB, 0.25, empty_rows=4)
+    csr = _mask_to_csr(mask, Hq, nB, cuda_dev)
+    ws = sa.Workspace(cuda_dev)
+    scale = 1 / math.sqrt(128)
+    out, lse = sa.sparse_prefill_attn(wl.cache.to(cuda_dev), wl.q.to(cuda_dev), csr, scale, ws=ws)
+    ws.raise_on_fault()
+    ref, ref_lse = oracle.prefill(wl.cache, wl.q, 64, mask, scale)
+    g_out = out.float().cpu().numpy().reshape(-1, 128)
+    g_lse = lse.cpu().numpy().reshape(-1)
+    assert_close_attn(g_out, ref)
+    fin = np.isfinite(ref_lse)
+    assert np.all(np.isneginf(g_lse[~fin])) and np.all(g_out[~fin] == 0)
+    np.testing.assert_allclose(g_lse[fin], ref_lse[fin], atol=2e-3, rtol=0)
+    seen = np.zeros((Hq, nB), dtype=np.int64)
+    G = Hq // Hkv
+    for h0, i0, h1, i1 in _schedule_items(ws, Hq, Hkv, nB):
+        assert 0 <= h0 < Hq and 0 <= i0 < nB
+        seen[h0, i0] += 1
+        if h1 >= 0:
+            assert 0 <= h1 < Hq and 0 <= i1 < nB and h0 // G == h1 // G
+            seen[h1, i1] += 1
+    assert np.array_equal(seen, np.ones((Hq, nB), dtype=np.int64))
