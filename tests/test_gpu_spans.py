@@ -97,7 +97,7 @@ def test_masked_decode_modes(cuda_dev, origin):
         want = _oracle_members(lens, Lmax, P, ref_spans)
         np.testing.assert_array_equal(got, want)
         ref, ref_lse = oracle.decode_members(cache, q, want, scale)
-        for S in (1, 8):
+        for S in (1, 8, 64):   # at 64, short lists leave most splits empty
             out, lse = sa.sparse_decode_attn(gc, q.to(cuda_dev), sel, scale, S, ws=ws)
             assert_close_attn(out.float().cpu().numpy().reshape(-1, d), ref)
             np.testing.assert_allclose(lse.cpu().numpy().reshape(-1), ref_lse, atol=2e-3, rtol=0)
@@ -156,10 +156,36 @@ def test_masked_decode_group_shapes(cuda_dev, d, Hq, Hkv, qdt):
     sel = sa.select_blocks_spans(gc, spans, cnt, rnd, ws=ws)
     mem = _members_from_blocks(sel.blocks.cpu().numpy(), sel.block_counts.cpu().numpy(), P, Lmax)
     ref, ref_lse = oracle.decode_members(cache, q, mem, scale)
-    for S in (1, 3, 8):
+    for S in (1, 3, 8, 37):
         out, lse = sa.sparse_decode_attn(gc, q.to(cuda_dev), sel, scale, S, ws=ws)
         assert_close_attn(out.float().cpu().numpy().reshape(-1, d), ref)
         np.testing.assert_allclose(lse.cpu().numpy().reshape(-1), ref_lse, atol=2e-3, rtol=0)
+    ws.raise_on_fault()
+
+
+@pytest.mark.parametrize("S", [1, 5, 64])
+def test_masked_decode_64_token_pages(cuda_dev, S):
+    """64-token pages: a split covers at least two list entries, so with many
+    splits most of them stay empty and the combine skips them."""
+    lens = [3000, 130, 6100]
+    P, d, Hq, Hkv = 64, 128, 16, 2
+    cache, q = W.random_decode(41 + S, len(lens), Hq, Hkv, d, lens, P)
+    Lmax = cache.max_pages * P
+    gc = cache.to(cuda_dev)
+    ws = sa.Workspace(cuda_dev)
+    scale = 1 / math.sqrt(d)
+    prod = [SP.spans_for(SP.FOCUS, lens[0], 2048, 7, [0, 1]), SP.spans_for(SP.STREAMING, lens[1], 2048),
+            SP.spans_for(SP.LOCAL, lens[2], 2048)]
+    spans, cnt, rnd = SP.pack(prod, cuda_dev)
+    sel = sa.select_blocks_spans(gc, spans, cnt, rnd, ws=ws)
+    mem = _members_from_blocks(sel.blocks.cpu().numpy(), sel.block_counts.cpu().numpy(), P, Lmax)
+    ref_spans = [OM.mode_spans(OM.FOCUS, lens[0], 2048, 7, [0, 1]), OM.mode_spans(OM.STREAM, lens[1], 2048),
+                 OM.mode_spans(OM.LOCAL, lens[2], 2048)]
+    np.testing.assert_array_equal(mem, _oracle_members(lens, Lmax, P, ref_spans))
+    ref, ref_lse = oracle.decode_members(cache, q, mem, scale)
+    out, lse = sa.sparse_decode_attn(gc, q.to(cuda_dev), sel, scale, S, ws=ws)
+    assert_close_attn(out.float().cpu().numpy().reshape(-1, d), ref)
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(-1), ref_lse, atol=2e-3, rtol=0)
     ws.raise_on_fault()
 
 
