@@ -13,7 +13,9 @@
 // Lanes are grouped by G = D/8: a group owns one token row at a time and each
 // lane holds 8 of its D elements (one 16-byte load of K and one of V).
 // Every group walks U consecutive list positions per step, so each lane has
-// 2U independent 16-byte loads in flight; the row is reduced over the group
+// 2U independent 16-byte loads in flight (for token lists the positions of a
+// window are first resolved to row offsets in shared memory, so those loads
+// wait on nothing else); the row is reduced over the group
 // with xor shuffles and folded into a per-group online softmax (base-2
 // exponentials on log2(e)-prescaled scores).  The groups' partial states are
 // merged through shared memory at the end.  The kernel is bound by the HBM
@@ -22,6 +24,8 @@
 
 namespace sa {
 namespace {
+
+constexpr int kStage = 1024;   // token-list positions resolved per window
 
 template <int D>
 struct DecodeCfg {
@@ -51,6 +55,7 @@ __global__ void __launch_bounds__(256) k_decode_split(const DecodeArgs a)
     constexpr int G = C::G, GPW = C::GPW, NG = C::NG;
     __shared__ float s_m[NG], s_l[NG];
     __shared__ float s_acc[NG * D];
+    __shared__ long long s_off[BLOCKS ? 1 : kStage];   // token lists: element offsets of a window's rows
 
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
     const int gl = lane & (G - 1);
@@ -121,56 +126,8 @@ __global__ void __launch_bounds__(256) k_decode_split(const DecodeArgs a)
     const int32_t *ptb = a.c.pt + (size_t)b * a.c.max_pages;
     const int Pm = (1 << a.c.Plog2) - 1;
 
-    // warp-uniform loop: every lane of a warp runs the same iterations
-    for (int base0 = lo + warp * GPW * U; base0 < hi; base0 += NG * U) {
-        const int base = base0 + sub * U;
-        uint4 kr[U], vr[U];
-        bool ok[U];
-        int e_idx = 0, e_off = 0;
-        int4 e_cur = make_int4(0, 0, 0, 0);
-        if (BLOCKS && base < hi) {
-            e_idx = locate_entry(ent, ne, base);
-            e_cur = ent[e_idx];
-            e_off = base - e_cur.w;
-        }
-#pragma unroll
-        for (int u = 0; u < U; ++u) {
-            const int pos = base + u;
-            ok[u] = pos < hi;
-            int t = 0;
-            if (ok[u]) {
-                if (!BLOCKS) {
-                    t = __ldg(a.idx + (size_t)row * a.kcap + pos);
-                } else {
-                    while (e_off >= e_cur.z - e_cur.y && e_idx + 1 < ne) {
-                        e_off -= e_cur.z - e_cur.y;
-                        e_cur = ent[++e_idx];
-                    }
-                    t = (e_cur.x << a.c.Plog2) + e_cur.y + e_off;
-                    ++e_off;
-                }
-                if (t < 0 || t >= L) {
-                    fault(st, CHK_INDEX, t);
-                    ok[u] = false;
-                }
-            }
-            int page = 0;
-            if (ok[u]) {
-                page = __ldg(ptb + (t >> a.c.Plog2));
-                if (page < 0 || page >= a.c.num_pages) {
-                    fault(st, CHK_PAGE, page);
-                    ok[u] = false;
-                }
-            }
-            const size_t off = ((((size_t)page * a.c.Hkv + g) << a.c.Plog2) + (t & Pm)) * D + gl * 8;
-            if (ok[u]) {
-                kr[u] = ldg_nc_v4(kbase + off);
-                vr[u] = ldg_nc_v4(vbase + off);
-            } else {
-                kr[u] = make_uint4(0, 0, 0, 0);
-                vr[u] = make_uint4(0, 0, 0, 0);
-            }
-        }
+    // the U rows of one step -> online softmax state of the group
+    auto consume = [&](const uint4 (&kr)[U], const uint4 (&vr)[U], const bool (&ok)[U]) {
         float sc[U];
 #pragma unroll
         for (int u = 0; u < U; ++u) {
@@ -209,6 +166,101 @@ __global__ void __launch_bounds__(256) k_decode_split(const DecodeArgs a)
                 acc[7] = fmaf(pw, bf_hi(vr[u].w), acc[7]);
             }
             m = mn;
+        }
+    };
+
+    if (!BLOCKS) {
+        // Token lists: the part's positions are resolved (index -> page ->
+        // element offset of the row, -1 if invalid) into shared memory a
+        // window at a time, so the main loop's loads depend on nothing but
+        // a shared-memory read.
+        for (int w0 = lo; w0 < hi; w0 += kStage) {
+            const int wn = min(kStage, hi - w0);
+            __syncthreads();   // the previous window has been consumed
+            for (int i = threadIdx.x; i < wn; i += blockDim.x) {
+                const int t = __ldg(a.idx + (size_t)row * a.kcap + w0 + i);
+                long long off = -1;
+                if (t < 0 || t >= L) {
+                    fault(st, CHK_INDEX, t);
+                } else {
+                    const int page = __ldg(ptb + (t >> a.c.Plog2));
+                    if (page < 0 || page >= a.c.num_pages)
+                        fault(st, CHK_PAGE, page);
+                    else
+                        off = (long long)(((((size_t)page * a.c.Hkv + g) << a.c.Plog2) + (t & Pm)) * D);
+                }
+                s_off[i] = off;
+            }
+            __syncthreads();
+            // warp-uniform loop: every lane of a warp runs the same iterations
+            for (int base0 = warp * GPW * U; base0 < wn; base0 += NG * U) {
+                const int base = base0 + sub * U;
+                uint4 kr[U], vr[U];
+                bool ok[U];
+#pragma unroll
+                for (int u = 0; u < U; ++u) {
+                    const int pos = base + u;
+                    const long long off = pos < wn ? s_off[pos] : -1;
+                    ok[u] = off >= 0;
+                    if (ok[u]) {
+                        kr[u] = ldg_nc_v4(kbase + off + gl * 8);
+                        vr[u] = ldg_nc_v4(vbase + off + gl * 8);
+                    } else {
+                        kr[u] = make_uint4(0, 0, 0, 0);
+                        vr[u] = make_uint4(0, 0, 0, 0);
+                    }
+                }
+                consume(kr, vr, ok);
+            }
+        }
+    } else {
+        // block lists: positions map to tokens through the entries
+        for (int base0 = lo + warp * GPW * U; base0 < hi; base0 += NG * U) {
+            const int base = base0 + sub * U;
+            uint4 kr[U], vr[U];
+            bool ok[U];
+            int e_idx = 0, e_off = 0;
+            int4 e_cur = make_int4(0, 0, 0, 0);
+            if (base < hi) {
+                e_idx = locate_entry(ent, ne, base);
+                e_cur = ent[e_idx];
+                e_off = base - e_cur.w;
+            }
+#pragma unroll
+            for (int u = 0; u < U; ++u) {
+                const int pos = base + u;
+                ok[u] = pos < hi;
+                int t = 0;
+                if (ok[u]) {
+                    while (e_off >= e_cur.z - e_cur.y && e_idx + 1 < ne) {
+                        e_off -= e_cur.z - e_cur.y;
+                        e_cur = ent[++e_idx];
+                    }
+                    t = (e_cur.x << a.c.Plog2) + e_cur.y + e_off;
+                    ++e_off;
+                    if (t < 0 || t >= L) {
+                        fault(st, CHK_INDEX, t);
+                        ok[u] = false;
+                    }
+                }
+                int page = 0;
+                if (ok[u]) {
+                    page = __ldg(ptb + (t >> a.c.Plog2));
+                    if (page < 0 || page >= a.c.num_pages) {
+                        fault(st, CHK_PAGE, page);
+                        ok[u] = false;
+                    }
+                }
+                const size_t off = ((((size_t)page * a.c.Hkv + g) << a.c.Plog2) + (t & Pm)) * D + gl * 8;
+                if (ok[u]) {
+                    kr[u] = ldg_nc_v4(kbase + off);
+                    vr[u] = ldg_nc_v4(vbase + off);
+                } else {
+                    kr[u] = make_uint4(0, 0, 0, 0);
+                    vr[u] = make_uint4(0, 0, 0, 0);
+                }
+            }
+            consume(kr, vr, ok);
         }
     }
 
