@@ -487,7 +487,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 // query blocks, so a window holds G * Wq <= 64 rows of the group.  A pair's
 // waste is |A xor B|, the key blocks listed by one row only, which the CTA
 // executes for both halves; rows are paired greedily, smallest waste first,
-// ties to the lowest pair index, then improved by 2-opt exchanges.  Wastes come from per-row bitmaps in shared
+// ties to the lowest pair index (as rounds of mutually-best pairs), then
+// improved by 2-opt exchanges.  Wastes come from per-row bitmaps in shared
 // memory (popcounts of xor), over chunks of kSchedBits key blocks.  One CTA
 // per (kv head, window); items are ordered kv-head-major, latest windows
 // first.
@@ -510,6 +511,8 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
     __shared__ int cost[kSchedPairs];
     __shared__ int red_c[8], red_p[8];
     __shared__ int pr_a[kSchedRows / 2], pr_b[kSchedRows / 2];
+    __shared__ int s_best[kSchedRows], s_taken;
+    __shared__ unsigned long long s_used;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nQB = (a.T + 63) >> 6;
     const int G = a.Hq / a.c.Hkv;
@@ -545,65 +548,59 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
             }
         }
     }
-    // greedy pairing = one pass over the pairs in ascending (waste, row a,
-    // row b) order, taking a pair when both rows are still free.  Keys
-    // (waste clamped to 20 bits, then the two 6-bit row ids) are bitonic-sorted
-    // in the bitmap's shared memory, which is free now.
-    uint32_t *keys = &bits[0][0];
-    constexpr int kKeys = 2048;   // >= kSchedPairs, power of two
-    static_assert(kKeys >= kSchedPairs && kKeys <= kSchedRows * (kSchedWords + 1), "key buffer");
+    // Greedy pairing (repeatedly take the free pair of smallest (waste, row,
+    // row) key), computed as rounds of locally dominant pairs: every free row
+    // finds its best free partner, and two rows that pick each other are
+    // paired.  Under a strict order on the pairs this takes exactly the pairs
+    // of the sequential greedy, and every round takes at least one (the
+    // smallest free pair).  Keys: waste clamped to 20 bits, then the two
+    // 6-bit row ids.
     __syncthreads();
-    for (int ka = warp; ka < kSchedRows; ka += 8) {
-        for (int kb = ka + 1 + lane; kb < kSchedRows; kb += 32) {
-            const int p = pair_index(ka, kb, kSchedRows);
-            uint32_t key = 0xFFFFFFFFu;
-            if (kb < nc) key = ((uint32_t)min(cost[pair_index(ka, kb, nc)], (1 << 20) - 1) << 12) | (ka << 6) | kb;
-            keys[p] = key;
-        }
-    }
-    for (int p = kSchedPairs + tid; p < kKeys; p += 256) keys[p] = 0xFFFFFFFFu;
-    for (int kk = 2; kk <= kKeys; kk <<= 1) {
-        for (int j = kk >> 1; j > 0; j >>= 1) {
-            __syncthreads();
-            for (int i = tid; i < kKeys; i += 256) {
-                const int ixj = i ^ j;
-                if (ixj > i) {
-                    const uint32_t x = keys[i], y = keys[ixj];
-                    const bool up = (i & kk) == 0;
-                    if ((x > y) == up) {
-                        keys[i] = y;
-                        keys[ixj] = x;
-                    }
-                }
-            }
-        }
+    if (tid == 0) {
+        s_used = 0ull;
+        s_taken = 0;
     }
     __syncthreads();
     const int base = g * nQB * (G / 2) + (nQB - i1) * (G / 2);
-    if (warp == 0) {
-        unsigned long long u = 0ull;
-        int t = 0;
-        for (int q0 = 0; q0 < np && t < nc / 2; q0 += 32) {
-            const uint32_t key = keys[q0 + lane];   // q0 + lane < kKeys; padding keys sort last
-            const int ka = (key >> 6) & 63, kb = key & 63;
-            const bool cand = q0 + lane < np && !(u >> ka & 1ull) && !(u >> kb & 1ull);
-            unsigned m = __ballot_sync(0xffffffffu, cand);
-            while (m) {
-                const int l = __ffs(m) - 1;
-                m &= m - 1;
-                const int xa = __shfl_sync(0xffffffffu, ka, l), xb = __shfl_sync(0xffffffffu, kb, l);
-                if (!(u >> xa & 1ull) && !(u >> xb & 1ull)) {
-                    u |= (1ull << xa) | (1ull << xb);
-                    if (lane == 0) {
-                        pr_a[t] = xa;
-                        pr_b[t] = xb;
-                    }
-                    ++t;
+    for (int round = 0; round < kSchedRows; ++round) {
+        const unsigned long long u = s_used;
+        if (s_taken >= nc / 2) break;   // uniform: read after a barrier
+        for (int ka = warp; ka < nc; ka += 8) {
+            uint32_t bk = 0xFFFFFFFFu;
+            if (!(u >> ka & 1ull)) {
+                for (int kb = lane; kb < nc; kb += 32) {
+                    if (kb == ka || (u >> kb & 1ull)) continue;
+                    const int lo = min(ka, kb), hi = max(ka, kb);
+                    const uint32_t key =
+                        ((uint32_t)min(cost[pair_index(lo, hi, nc)], (1 << 20) - 1) << 12) | (lo << 6) | hi;
+                    bk = min(bk, key);
                 }
             }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) bk = min(bk, __shfl_xor_sync(0xffffffffu, bk, o));
+            if (lane == 0) {
+                const int lo = (bk >> 6) & 63, hi = bk & 63;
+                s_best[ka] = bk == 0xFFFFFFFFu ? -1 : (lo == ka ? hi : lo);
+            }
         }
+        __syncthreads();
+        if (tid == 0) {
+            unsigned long long nu = u;
+            int t = s_taken;
+            for (int x = 0; x < nc; ++x) {
+                const int y = s_best[x];
+                if (y > x && !(u >> x & 1ull) && s_best[y] == x) {
+                    pr_a[t] = x;
+                    pr_b[t] = y;
+                    ++t;
+                    nu |= (1ull << x) | (1ull << y);
+                }
+            }
+            s_used = nu;
+            s_taken = t;
+        }
+        __syncthreads();
     }
-    __syncthreads();
     // 2-opt: repeatedly apply the exchange of partners between two pairs that
     // lowers the total waste most (ties to the lowest pair of pairs), until
     // none does
