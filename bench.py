@@ -51,6 +51,14 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 LAUNCHES = {"select_topk": 2, "decode": 2, "spans": 1, "rbs_explicit": 7, "prefill": 2}
 
 
+def pct(xs, q):
+    """q-th percentile (nearest rank) of per-step device times, ms (this rank)."""
+    if not xs:
+        return None
+    v = sorted(xs)
+    return round(v[min(len(v) - 1, max(0, math.ceil(q / 100 * len(v)) - 1))], 4)
+
+
 def peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -387,6 +395,10 @@ def main():
     tiered = tiered_measure(msk, cfg, dev)
     total_ms = t_start.elapsed_time(t_end)
     parts = {"decode": 0.0, "masked": 0.0, "rbs_select": 0.0, "prefill": 0.0}
+    per_step = {"decode": [], "prefill": []}
+    for e in evs:
+        per_step["decode"].append(e[0].elapsed_time(e[1]))
+        per_step["prefill"].append(e[3].elapsed_time(e[4]))
     for e in evs:
         parts["decode"] += e[0].elapsed_time(e[1])
         parts["masked"] += e[1].elapsed_time(e[2])
@@ -424,10 +436,12 @@ def main():
                          % (cfg.dec["B"] * cfg.dec["Hkv"] * cfg.dec["L"] * 256 / 1e9, T * Hqp * dp * 2 / 1e9)},
         "decode": {"gbs": round(dec_gbs, 2), "frac_hbm": round(per_gpu_dec / pk["hbm_gbs"], 4),
                    "ms_per_group": round(dec_ms / K, 4), "bytes_per_group": dec_bytes,
+                   "ms_p50": pct(per_step["decode"], 50), "ms_p95": pct(per_step["decode"], 95),
                    "tokens_per_s": round(world * K * cfg.dec["B"] / (dec_ms * 1e-3), 1)},
         "prefill": {"tflops": round(pre_tflops, 2), "frac_bf16_sustained": round(per_gpu_pre / pk["bf16_tflops_sustained"], 4),
                     "frac_bf16_burst": round(per_gpu_pre / pk["bf16_tflops"], 4),
-                    "ms": round(pre_ms / K, 4), "selected_tiles": sel_tiles,
+                    "ms": round(pre_ms / K, 4), "ms_p50": pct(per_step["prefill"], 50),
+                    "ms_p95": pct(per_step["prefill"], 95), "selected_tiles": sel_tiles,
                     "executed_tiles_64x64": exec_tiles,
                     "executed_tflops": round(world * K * exec_tiles * TILE_FLOPS / (pre_ms * 1e-3) / 1e12, 2),
                     "tokens_per_s": round(world * K * T / (pre_ms * 1e-3), 1)},
@@ -747,7 +761,26 @@ def cpu_baseline(cfg, dec, pre, pc, pr, budget_s=10.0):
         sel = mask[0, i * (i + 1) // 2: i * (i + 1) // 2 + i + 1]
         keys = sum(min(64, int(t) - 64 * int(j) + 1) for j in np.nonzero(sel)[0])
         flops += 4 * keys * 128
+    # one thread on a fixed small unit: kv head 0's query heads of sequence 0
+    # (anchor top-k + the decode layers)
+    cache1, vs1, qs1 = _sub_decode(dec, [0])
+    G = c["Hq"] // c["Hkv"]
+    import torch
+    def head0(t):   # [pages][Hkv][P][d] -> kv head 0 only
+        return t[:, :1].contiguous()
+    from sparse_attention_aware_b200 import workloads as W
+    c1 = W.PagedCache(head0(cache1.k), head0(vs1[0]), cache1.page_table, cache1.seq_lens)
+    q1 = [q[:, :G].contiguous() for q in qs1]
+    t2 = time.time()
+    idx1, cnt1 = oracle.select_topk(oracle.CacheView(c1), q1[0], c["k"], nthreads=1)
+    for li in range(c["layers"]):
+        oracle.decode_tokens(oracle.CacheView(c1.with_v(head0(vs1[li]))), q1[li], idx1, cnt1, scale, nthreads=1)
+    t_one = time.time() - t2
+    one_bytes = decode_group_bytes(dict(c, B=1, Hq=G, Hkv=1))
     return {"value": round(dec_gbs, 4), "unit": "GB/s", "cores": oracle.threads(), "kind": "oracle",
+            "single_thread": {"value": round(one_bytes / t_one / 1e9, 4), "unit": "GB/s", "seconds": round(t_one, 2),
+                              "sample": "anchor top-k + %d layers, sequence 0, kv head 0 and its %d query heads"
+                                        % (c["layers"], G)},
             "sample": "decode: anchor top-k + %d layers for %d of %d sequences (all %d heads), %.1f s; "
                       "prefill: RBS selection for 1 head + 256 sampled query rows, %.1f s"
                       % (c["layers"], nseq, c["B"], c["Hq"], t_dec, t_pre),
