@@ -143,11 +143,16 @@ class ClockSampler:
         self.bus_id = str(bus_id or "").lower()
         self.proc = None
         self.lines = []
+        self.first = 0
+
+    def mark(self):
+        """Samples read before this call (the warm-up pause) are not used."""
+        self.first = len(self.lines)
 
     def start(self):
         try:
             self.proc = subprocess.Popen(["nvidia-smi", "--query-gpu=" + self.Q, "--format=csv,noheader,nounits",
-                                          "-lms", "200"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
+                                          "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL,
                                          text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -168,7 +173,8 @@ class ClockSampler:
             self.proc.kill()
         self.t.join(timeout=2)
         rows = []
-        for ln in self.lines:
+        lines = self.lines[self.first:] or self.lines
+        for ln in lines:
             f = [x.strip() for x in ln.split(",")]
             if len(f) < 10:
                 continue
@@ -372,6 +378,7 @@ def main():
     torch.cuda.synchronize()
     t_start, t_end = ev(), ev()
     evs = []
+    clocks.mark()
     t_start.record(stream)
     for _ in range(args.steps):
         run_step(evs)
