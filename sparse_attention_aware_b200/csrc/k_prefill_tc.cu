@@ -601,6 +601,24 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
         }
         __syncthreads();
     }
+    if (tid == 0 && s_taken < nc / 2) {
+        // not reached (every round takes the smallest free pair); kept so that
+        // every row is in an item whatever happens above
+        int t = s_taken, prev = -1;
+        for (int x = 0; x < nc; ++x) {
+            if (s_used >> x & 1ull) continue;
+            if (prev < 0) {
+                prev = x;
+            } else {
+                pr_a[t] = prev;
+                pr_b[t] = x;
+                ++t;
+                prev = -1;
+            }
+        }
+        s_taken = t;
+    }
+    __syncthreads();
     // 2-opt: repeatedly apply the exchange of partners between two pairs that
     // lowers the total waste most (ties to the lowest pair of pairs), until
     // none does
