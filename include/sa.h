@@ -311,9 +311,11 @@ SA_API sa_status sa_sparse_decode_attn_noalloc(const sa_kv_cache *kv, const void
  *   lse_out  fp32 [num_tokens][num_q_heads] natural log, nullable
  *   causal   must be 1; scale must be finite and > 0.
  * Work is scheduled in pairs of 64-row query blocks that share their K/V
- * tiles (two heads of one GQA group at the same query block, matched greedily
- * by the overlap of their CSR rows; adjacent query blocks of one head when
- * the group size is odd); the pairing list lives in the workspace.
+ * tiles: two (head, query block) rows of one GQA group from a window of
+ * 64/G nearby query blocks, matched greedily by the key blocks the two rows
+ * do not share and refined by pair exchanges (adjacent query blocks of one
+ * head when the group size is odd or above 16); the pairing list lives in
+ * the workspace.  Results do not depend on the pairing.
  */
 SA_API sa_status sa_sparse_prefill_attn(const sa_kv_cache *kv, const void *q, int32_t num_q_heads,
                                  int32_t num_tokens, const sa_block_list *csr, float scale,
