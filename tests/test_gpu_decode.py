@@ -64,6 +64,24 @@ def test_decode_tokens_random(cuda_dev, d, P, qdt, Hq, Hkv, splits):
     assert torch.equal(out, out2) and torch.equal(lse, lse2)
 
 
+@pytest.mark.parametrize("splits", [1, 2])
+def test_decode_tokens_long_parts(cuda_dev, splits):
+    """Parts longer than the 1024 positions a decode CTA resolves into shared
+    memory at a time (up to 3000 positions in one part: three windows)."""
+    lens = [5000, 2500, 3100]
+    cache, q = W.random_decode(23 + splits, len(lens), 8, 2, 128, lens, 16)
+    idx, cnt = _random_idx(9 + splits, len(lens), 8, 3000, lens, [3000, 2047, 1025, 1])
+    scale = 1 / math.sqrt(128)
+    ref, ref_lse = oracle.decode_tokens(cache, q, idx, cnt, scale)
+    gc = cache.to(cuda_dev)
+    sel = sa.TokenSelection(torch.from_numpy(idx).to(cuda_dev), torch.from_numpy(cnt).to(cuda_dev))
+    ws = sa.Workspace(cuda_dev)
+    out, lse = sa.sparse_decode_attn(gc, q.to(cuda_dev), sel, scale, splits, ws=ws)
+    ws.raise_on_fault()
+    assert_close_attn(out.float().cpu().numpy().reshape(-1, 128), ref)
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(-1), ref_lse, atol=2e-3, rtol=0)
+
+
 def test_decode_split_invariance(cuda_dev):
     cache, q = W.random_decode(3, 2, 8, 2, 128, [2000, 999], 16)
     idx, cnt = _random_idx(1, 2, 8, 1024, [2000, 999], [1024, 900, 33])
