@@ -208,3 +208,35 @@ def test_prefill_group_sizes_and_schedule(cuda_dev, T, Hq, Hkv):
             assert 0 <= h1 < Hq and 0 <= i1 < nB and h0 // G == h1 // G
             seen[h1, i1] += 1
     assert np.array_equal(seen, np.ones((Hq, nB), dtype=np.int64))
+
+
+def test_prefill_longer_than_one_bitmap_chunk(cuda_dev):
+    """140000 tokens (2188 query blocks): the pairing windows near the end
+    build their row bitmaps in two chunks of 2048 key blocks.  Sparse random
+    mask (diagonal forced), sampled rows against the oracle, and the work
+    items still cover every row once."""
+    T, Hq, Hkv = 140000, 2, 1
+    wl = W.random_prefill(901, T, Hq, Hkv, 128, 64)
+    nB = (T + 63) // 64
+    rng = np.random.default_rng(17)
+    nP = nB * (nB + 1) // 2
+    mask = (rng.random((Hq, nP)) < 0.01).astype(np.uint8)
+    for i in range(nB):
+        mask[:, i * (i + 1) // 2 + i] = 1
+    ts = np.concatenate([[0, 131071, 131072, 139999, T - 64], rng.integers(0, T, 120)])
+    hs = rng.integers(0, Hq, len(ts))
+    rows = (ts * Hq + hs).astype(np.int64)
+    csr = _mask_to_csr(mask, Hq, nB, cuda_dev)
+    ws = sa.Workspace(cuda_dev)
+    scale = 1 / math.sqrt(128)
+    out, lse = sa.sparse_prefill_attn(wl.cache.to(cuda_dev), wl.q.to(cuda_dev), csr, scale, ws=ws)
+    ws.raise_on_fault()
+    ref, ref_lse = oracle.prefill(wl.cache, wl.q, 64, mask, scale, rows=rows)
+    assert_close_attn(out.float().cpu().numpy().reshape(-1, 128)[rows], ref)
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(-1)[rows], ref_lse, atol=2e-3, rtol=0)
+    seen = np.zeros((Hq, nB), dtype=np.int64)
+    for h0, i0, h1, i1 in _schedule_items(ws, Hq, Hkv, nB):
+        seen[h0, i0] += 1
+        if h1 >= 0:
+            seen[h1, i1] += 1
+    assert np.array_equal(seen, np.ones((Hq, nB), dtype=np.int64))
