@@ -160,3 +160,53 @@ def test_binding_fails_loudly_without_library(tmp_path):
             L.load(str(tmp_path / "missing.so"))
     finally:
         L._lib = saved
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include <string.h>
+#include "sa.h"
+
+int main(void)
+{
+    if (sa_version() < 100) return 1;
+    if (strncmp(sa_status_string(SA_OK), "SA_OK", 5) != 0) return 2;
+    if (strncmp(sa_status_string(SA_ERR_WORKSPACE), "SA_ERR_WORKSPACE", 16) != 0) return 3;
+    sa_kv_cache kv;
+    memset(&kv, 0, sizeof kv);
+    kv.k = (const void *)0x10000;
+    kv.v = (const void *)0x20000;
+    kv.page_table = (const int32_t *)0x30000;
+    kv.seq_lens = (const int32_t *)0x40000;
+    kv.batch = 2;
+    kv.num_kv_heads = 2;
+    kv.head_dim = 128;
+    kv.page_size = 16;
+    kv.max_pages_per_seq = 8;
+    kv.num_pages = 16;
+    sa_ws_query q;
+    memset(&q, 0, sizeof q);
+    q.num_q_heads = 8;
+    q.k = 16;
+    if (sa_workspace_bytes(SA_OP_SELECT_TOPK, &kv, &q) != 256 + 2 * 8 * 8 * 16 * 4) return 4;
+    kv.head_dim = 96;
+    if (sa_workspace_bytes(SA_OP_SELECT_TOPK, &kv, &q) != 0) return 5;
+    puts("ok");
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    """include/sa.h compiles as C99 with no CUDA header, and a C program links
+    libsa.so and calls its host-only entry points."""
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    libdir = os.path.dirname(L.LIB_PATH)
+    inc = os.path.dirname(HEADER)
+    import subprocess
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-pedantic", "-I", inc, str(src), "-o", str(exe),
+                    "-L", libdir, "-l:libsa.so", "-Wl,-rpath," + libdir], check=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True)
+    assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
