@@ -9,6 +9,7 @@ from __future__ import annotations
 
 import ctypes
 import dataclasses
+import functools
 import math
 from typing import Optional, Sequence
 
@@ -39,6 +40,23 @@ def _ptr(t: Optional[torch.Tensor]):
 def _stream(stream=None):
     s = stream if stream is not None else torch.cuda.current_stream()
     return ctypes.c_void_p(s.cuda_stream)
+
+
+def _on_call_stream(fn):
+    """When an entry point is given ``stream=``, the tensors it makes itself
+    (contiguous copies of inputs, threshold tensors, default outputs, a
+    growing workspace) are made on that stream, so that they are ordered
+    before the kernels that read them and the caching allocator does not hand
+    their memory out again while those kernels run.  Without ``stream=`` the
+    call runs on torch's current stream as before."""
+    @functools.wraps(fn)
+    def call(*args, **kw):
+        s = kw.get("stream")
+        if s is None:
+            return fn(*args, **kw)
+        with torch.cuda.stream(s):
+            return fn(*args, **kw)
+    return call
 
 
 def kv_struct(cache) -> L.KVCacheS:
@@ -154,6 +172,7 @@ class BlockCSR:
 # --------------------------------------------------------------------------
 # entry points
 # --------------------------------------------------------------------------
+@_on_call_stream
 def select_topk(cache, q: torch.Tensor, k: int, idx: Optional[torch.Tensor] = None,
                 count: Optional[torch.Tensor] = None, ws: Optional[Workspace] = None,
                 stream=None) -> TokenSelection:
@@ -172,6 +191,7 @@ def select_topk(cache, q: torch.Tensor, k: int, idx: Optional[torch.Tensor] = No
     return TokenSelection(idx, count)
 
 
+@_on_call_stream
 def sparse_decode_attn(cache, q: torch.Tensor, sel, scale: Optional[float] = None, num_splits: int = 1,
                        out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                        want_lse: bool = True, ws: Optional[Workspace] = None, stream=None):
@@ -193,6 +213,7 @@ def sparse_decode_attn(cache, q: torch.Tensor, sel, scale: Optional[float] = Non
     return out, lse
 
 
+@_on_call_stream
 def fetch_pages(host_k: torch.Tensor, host_v: torch.Tensor, dev_k: torch.Tensor, dev_v: torch.Tensor,
                 pairs: torch.Tensor, ws: Optional[Workspace] = None, stream=None) -> None:
     """Copy host-tier pages into device page slots (``sa_fetch_pages``).
@@ -215,6 +236,7 @@ def fetch_pages(host_k: torch.Tensor, host_v: torch.Tensor, dev_k: torch.Tensor,
                                    wp, wn, _stream(stream)), "sa_fetch_pages")
 
 
+@_on_call_stream
 def select_blocks_spans(cache, spans: torch.Tensor, span_counts: torch.Tensor, span_round: torch.Tensor,
                         max_blocks: Optional[int] = None, out: Optional[BlockSelection] = None,
                         ws: Optional[Workspace] = None, stream=None) -> BlockSelection:
@@ -240,6 +262,7 @@ def select_blocks_spans(cache, spans: torch.Tensor, span_counts: torch.Tensor, s
     return out
 
 
+@_on_call_stream
 def select_blocks_rbs(cache, q: torch.Tensor, block_size: int = 64, scale: Optional[float] = None,
                       tau_c=None, tau_r=None, p_c: float = 0.95, p_r: float = 0.97,
                       force_diag: bool = True, force_first: bool = True,
@@ -280,6 +303,7 @@ def select_blocks_rbs(cache, q: torch.Tensor, block_size: int = 64, scale: Optio
     return out
 
 
+@_on_call_stream
 def sparse_prefill_attn(cache, q: torch.Tensor, csr: BlockCSR, scale: Optional[float] = None,
                         out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None,
                         want_lse: bool = True, ws: Optional[Workspace] = None, stream=None):

@@ -210,3 +210,21 @@ def test_header_is_plain_c_and_links(lib, tmp_path):
                     "-L", libdir, "-l:libsa.so", "-Wl,-rpath," + libdir], check=True)
     r = subprocess.run([str(exe)], capture_output=True, text=True)
     assert r.returncode == 0 and r.stdout.strip() == "ok", (r.returncode, r.stdout, r.stderr)
+
+
+def test_binding_stream_wrapper_passes_calls_through():
+    """Without ``stream=`` an entry point runs exactly as written; the wrapper
+    keeps names and docstrings (it only enters the given stream's context)."""
+    from sparse_attention_aware_b200 import api
+
+    @api._on_call_stream
+    def f(a, b=2, stream=None):
+        """doc"""
+        return a, b, stream
+
+    assert f(1) == (1, 2, None) and f(1, b=3, stream=None) == (1, 3, None)
+    assert f.__name__ == "f" and f.__doc__ == "doc"
+    for name in ("select_topk", "sparse_decode_attn", "select_blocks_spans", "select_blocks_rbs",
+                 "sparse_prefill_attn", "fetch_pages"):
+        fn = getattr(api, name)
+        assert fn.__name__ == name and fn.__wrapped__ is not None
