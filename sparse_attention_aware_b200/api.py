@@ -129,6 +129,20 @@ def workspace_bytes(op: int, cache, num_q_heads=0, k=0, num_splits=0, num_tokens
     return n
 
 
+def _need(t: torch.Tensor, shape, dtype, device, what: str) -> None:
+    """A caller-provided output (or index) tensor must have exactly the layout
+    the library writes: shape, dtype, contiguity and device."""
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous() or t.device != device:
+        raise ValueError("%s: need a contiguous %s tensor of shape %s on %s, got %s %s on %s"
+                         % (what, dtype, tuple(shape), device, t.dtype, tuple(t.shape), t.device))
+
+
+def _bf16_q(q: torch.Tensor, what: str) -> torch.Tensor:
+    if q.dtype != torch.bfloat16:
+        raise TypeError("%s: q must be bf16, got %s" % (what, q.dtype))
+    return q.contiguous()
+
+
 def _qdtype(q: torch.Tensor) -> int:
     if q.dtype == torch.float32:
         return L.DTYPE_F32
@@ -181,8 +195,10 @@ def select_topk(cache, q: torch.Tensor, k: int, idx: Optional[torch.Tensor] = No
     dev = q.device
     if idx is None:
         idx = torch.empty((B, Hq, k), dtype=torch.int32, device=dev)
+    _need(idx, (B, Hq, k), torch.int32, dev, "select_topk idx")
     if count is None:
         count = torch.empty((B, Hq), dtype=torch.int32, device=dev)
+    _need(count, (B, Hq), torch.int32, dev, "select_topk count")
     kv = kv_struct(cache)
     w = _ws(ws, dev)
     wp, wn = w.aligned(workspace_bytes(L.OP_SELECT_TOPK, cache, num_q_heads=Hq, k=k))
@@ -201,8 +217,11 @@ def sparse_decode_attn(cache, q: torch.Tensor, sel, scale: Optional[float] = Non
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     if out is None:
         out = torch.empty((B, Hq, d), dtype=torch.bfloat16, device=dev)
+    _need(out, (B, Hq, d), torch.bfloat16, dev, "sparse_decode_attn out")
     if lse is None and want_lse:
         lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _need(lse, (B, Hq), torch.float32, dev, "sparse_decode_attn lse")
     kv = kv_struct(cache)
     s = sel.struct()
     w = _ws(ws, dev)
@@ -248,6 +267,14 @@ def select_blocks_spans(cache, spans: torch.Tensor, span_counts: torch.Tensor, s
         mb = max_blocks if max_blocks is not None else cache.page_table.shape[1] + spans.shape[1]
         out = BlockSelection(torch.empty((B, mb, 4), dtype=torch.int32, device=dev),
                              torch.empty((B,), dtype=torch.int32, device=dev))
+    _need(out.blocks, (B, out.blocks.shape[1], 4), torch.int32, dev, "select_blocks_spans out.blocks")
+    _need(out.block_counts, (B,), torch.int32, dev, "select_blocks_spans out.block_counts")
+    S = spans.shape[1]
+    _need(spans, (B, S, 2), torch.int32, dev, "select_blocks_spans spans")
+    _need(span_counts, (B,), torch.int32, dev, "select_blocks_spans span_counts")
+    if span_round.dtype == torch.bool:
+        span_round = span_round.to(torch.uint8)
+    _need(span_round, (B, S), torch.uint8, dev, "select_blocks_spans span_round")
     kv = kv_struct(cache)
     a = L.BlockSelectArgsS()
     a.mode = L.SEL_SPANS
@@ -273,6 +300,7 @@ def select_blocks_rbs(cache, q: torch.Tensor, block_size: int = 64, scale: Optio
     otherwise quantile mode with p_c / p_r."""
     T, Hq, d = q.shape
     dev = q.device
+    q = _bf16_q(q, "select_blocks_rbs")
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     nB = (T + block_size - 1) // block_size
     if out is None:
@@ -280,6 +308,9 @@ def select_blocks_rbs(cache, q: torch.Tensor, block_size: int = 64, scale: Optio
         out = BlockCSR(torch.empty(Hq * nB + 1, dtype=torch.int32, device=dev),
                        torch.empty(max(cap, 1), dtype=torch.int32, device=dev),
                        torch.empty((2, Hq), dtype=torch.float32, device=dev), Hq, nB)
+    _need(out.row_ptr, (Hq * nB + 1,), torch.int32, dev, "select_blocks_rbs out.row_ptr")
+    _need(out.cols, (out.cols.numel(),), torch.int32, dev, "select_blocks_rbs out.cols")
+    _need(out.tau, (2, Hq), torch.float32, dev, "select_blocks_rbs out.tau")
     tc = tr = None
     if tau_c is not None:
         tc = torch.as_tensor(tau_c, dtype=torch.float32, device=dev).expand(Hq).contiguous()
@@ -310,11 +341,18 @@ def sparse_prefill_attn(cache, q: torch.Tensor, csr: BlockCSR, scale: Optional[f
     """Causal block-sparse prefill (``sa_sparse_prefill_attn``).  Returns (out bf16, lse fp32)."""
     T, Hq, d = q.shape
     dev = q.device
+    q = _bf16_q(q, "sparse_prefill_attn")
     scale = 1.0 / math.sqrt(d) if scale is None else scale
     if out is None:
         out = torch.empty((T, Hq, d), dtype=torch.bfloat16, device=dev)
+    _need(out, (T, Hq, d), torch.bfloat16, dev, "sparse_prefill_attn out")
     if lse is None and want_lse:
         lse = torch.empty((T, Hq), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _need(lse, (T, Hq), torch.float32, dev, "sparse_prefill_attn lse")
+    nQB = (T + 63) // 64
+    _need(csr.row_ptr, (Hq * nQB + 1,), torch.int32, dev, "sparse_prefill_attn csr.row_ptr")
+    _need(csr.cols, (csr.cols.numel(),), torch.int32, dev, "sparse_prefill_attn csr.cols")
     kv = kv_struct(cache)
     c = L.BlockListS()
     c.row_ptr, c.cols, c.nnz_capacity = csr.row_ptr.data_ptr(), csr.cols.data_ptr(), csr.cols.numel()

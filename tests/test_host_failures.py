@@ -47,3 +47,30 @@ def test_small_or_misaligned_workspace_is_rejected_before_launch():
     # too small by one byte, and misaligned: host checks fail, nothing is launched
     assert lib.sa_select_topk(ctypes.byref(kv), qa.data_ptr(), L.DTYPE_F32, 4, 8, ia, ca, base, need - 1, None) == WS
     assert lib.sa_select_topk(ctypes.byref(kv), qa.data_ptr(), L.DTYPE_F32, 4, 8, ia, ca, base + 8, need, None) == WS
+
+
+def test_caller_tensors_with_the_wrong_layout_are_rejected_before_launch():
+    """Outputs the caller provides must have the exact layout the library
+    writes; the RBS selection and the prefill take bf16 queries only."""
+    cache, q = _cache()                       # B=1, Hq=4, d=64
+    with pytest.raises(ValueError, match="select_topk idx"):
+        sa.select_topk(cache, q, 8, idx=torch.zeros((1, 4, 9), dtype=torch.int32))
+    with pytest.raises(ValueError, match="select_topk count"):
+        sa.select_topk(cache, q, 8, count=torch.zeros((1, 4), dtype=torch.int64))
+    idx = torch.zeros((1, 4, 8), dtype=torch.int32)
+    sel = sa.TokenSelection(idx, torch.zeros((1, 4), dtype=torch.int32))
+    with pytest.raises(ValueError, match="sparse_decode_attn out"):
+        sa.sparse_decode_attn(cache, q, sel, 0.1, 2, out=torch.zeros((1, 4, 64), dtype=torch.float32))
+    with pytest.raises(ValueError, match="sparse_decode_attn lse"):
+        sa.sparse_decode_attn(cache, q, sel, 0.1, 2, lse=torch.zeros((4, 1), dtype=torch.float32))
+    wl = W.random_prefill(5, 200, 2, 1, 128, 64)
+    with pytest.raises(TypeError, match="bf16"):
+        sa.select_blocks_rbs(wl.cache, wl.q.float(), 64, tau_c=0.0, tau_r=0.0)
+    csr = sa.BlockCSR(torch.zeros(2 * 4 + 1, dtype=torch.int32), torch.zeros(8, dtype=torch.int32),
+                      torch.zeros((2, 2)), 2, 4)
+    with pytest.raises(TypeError, match="bf16"):
+        sa.sparse_prefill_attn(wl.cache, wl.q.float(), csr)
+    with pytest.raises(ValueError, match="csr.row_ptr"):
+        sa.sparse_prefill_attn(wl.cache, wl.q, sa.BlockCSR(torch.zeros(5, dtype=torch.int32), csr.cols, csr.tau, 2, 4))
+    with pytest.raises(ValueError, match="sparse_prefill_attn out"):
+        sa.sparse_prefill_attn(wl.cache, wl.q, csr, out=torch.zeros((200, 2, 128), dtype=torch.bfloat16)[:, :1])
