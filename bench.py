@@ -340,6 +340,11 @@ def main():
     torch.cuda.synchronize()
     sel_tiles = int(csr.row_ptr[-1])
     exec_tiles = 2 * union_tiles(csr, pre.q.shape[1], step.nB, step.ws[3])
+    # rows the query heads of each GQA group select, as a union (measured on
+    # the anchor's top-k sets of this workload)
+    step.decode_group(dec.q_layers)
+    torch.cuda.synchronize()
+    uni_mean, head_mean, uni_total = group_union_rows(step.idx, step.cnt, cfg.dec["Hkv"])
 
     stream = torch.cuda.current_stream()
     ev = lambda: torch.cuda.Event(enable_timing=True)
@@ -419,6 +424,10 @@ def main():
         [total_ms, parts["decode"], parts["masked"], parts["rbs_select"], parts["prefill"]], dev)
 
     dec_bytes = decode_group_bytes(cfg.dec)
+    # the same group counted with each (sequence, kv head)'s union of the
+    # heads' rows read once per layer instead of once per query head
+    union_bytes = dec_bytes - cfg.dec["layers"] * (cfg.dec["B"] * cfg.dec["Hq"] * cfg.dec["k"] - uni_total) \
+        * 2 * cfg.dec["d"] * 2
     m = cfg.msk
     msk_bytes = sum(step.masked_tokens[s % len(step.masked_tokens)] for s in range(K)) * m["Hkv"] * m["d"] * 2 * 2 \
         + K * 2 * m["B"] * m["Hq"] * m["d"] * 2
@@ -445,6 +454,9 @@ def main():
                    "l2": "inputs larger than L2 (decode K cache %.1f GB, prefill Q %.2f GB)"
                          % (cfg.dec["B"] * cfg.dec["Hkv"] * cfg.dec["L"] * 256 / 1e9, T * Hqp * dp * 2 / 1e9)},
         "decode": {"gbs": round(dec_gbs, 2), "frac_hbm": round(per_gpu_dec / pk["hbm_gbs"], 4),
+                   "union_rows_per_group": round(uni_mean, 1), "per_head_rows_per_group": round(head_mean, 1),
+                   "union_bytes_per_group": union_bytes, "union_gbs": round(world * K * union_bytes / (dec_ms * 1e-3) / 1e9, 2),
+                   "union_frac_hbm": round(K * union_bytes / (dec_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                    "ms_per_group": round(dec_ms / K, 4), "bytes_per_group": dec_bytes,
                    "ms_p50": pct(per_step["decode"], 50), "ms_p95": pct(per_step["decode"], 95),
                    "tokens_per_s": round(world * K * cfg.dec["B"] / (dec_ms * 1e-3), 1)},
@@ -465,9 +477,10 @@ def main():
                           "da_state_host_us_per_step": round(da_us, 2)},
         "tiered_kv": tiered,
         "roofline": {"bound": "tensor", "kernel": "k_prefill_tc", "achieved": round(per_gpu_pre, 2),
-                     "peak": pk["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                     "frac": round(per_gpu_pre / pk["bf16_tflops_sustained"], 4), "traffic": None,
-                     "peak_source": "%s bf16_tflops_sustained (kernel timed inside a multi-kernel step)" % pk_kind,
+                     "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": round(per_gpu_pre / pk["bf16_tflops"], 4), "traffic": None,
+                     "peak_source": "%s bf16_tflops (burst: the step lasts milliseconds and the timed region "
+                                    "well under a second)" % pk_kind,
                      "algorithmic": "selected tiles x 4*64*64*128 FLOP per launch; CUDA events around the launch"},
         "roofline_decode": {"bound": "hbm", "kernel": "k_topk_score + k_decode_split + combine",
                             "achieved": round(per_gpu_dec, 2), "peak": pk["hbm_gbs"], "unit": "GB/s",
@@ -633,7 +646,7 @@ def union_tiles(csr, Hq, nB, ws):
     cols = csr.cols[: int(rp[-1])].cpu().numpy()
     buf = ws.buf
     off = (-buf.data_ptr()) % 256 + 256
-    n_items = (buf.numel() - off) // 16
+    n_items = (Hq // 2) * nB          # even GQA groups of <= 16 heads (the bench's 32/4)
     items = buf[off: off + 16 * n_items].view(torch.int32).reshape(-1, 4).cpu().numpy()
     tot = 0
     for h0, i0, h1, i1 in items:
@@ -646,6 +659,26 @@ def union_tiles(csr, Hq, nB, ws):
         else:
             tot += len(a)
     return int(tot)
+
+
+def group_union_rows(idx, cnt, Hkv):
+    """Distinct selected rows per (sequence, kv head): the union of the top-k
+    sets of the group's query heads (each head selects on its own; the group
+    reads one K/V stream).  Returns (mean union rows per group, mean per-head
+    rows per group, total union rows)."""
+    import torch
+    B, Hq, k = idx.shape
+    G = Hq // Hkv
+    pos = torch.arange(k, device=idx.device)
+    valid = pos[None, None, :] < cnt[:, :, None]
+    big = torch.iinfo(torch.int32).max
+    x = torch.where(valid, idx, torch.full_like(idx, big)).reshape(B, Hkv, G * k)
+    x, _ = torch.sort(x, dim=-1)
+    new = torch.ones_like(x, dtype=torch.bool)
+    new[..., 1:] = x[..., 1:] != x[..., :-1]
+    uni = (new & (x != big)).sum(dim=-1)
+    per_head = cnt.reshape(B, Hkv, G).sum(dim=-1)
+    return float(uni.float().mean()), float(per_head.float().mean()), int(uni.sum())
 
 
 def e2e(step, dec, pre, msk, cfg, args, world, dev, dist):

@@ -59,34 +59,63 @@ def _on_call_stream(fn):
     return call
 
 
-def kv_struct(cache) -> L.KVCacheS:
+def kv_struct(cache, device=None) -> L.KVCacheS:
     """``cache``: any object with k, v, page_table, seq_lens tensors on the GPU
     (k/v bf16 [num_pages][Hkv][P][d], page_table int32 [B][max_pages],
-    seq_lens int32 [B])."""
+    seq_lens int32 [B]).  ``device``: when given, every cache tensor must be on
+    it (the device of the call's queries).  Raises ValueError otherwise."""
     k, v = cache.k, cache.v
-    assert k.dtype == torch.bfloat16 and v.dtype == torch.bfloat16
-    assert k.is_contiguous() and v.is_contiguous() and k.shape == v.shape
     pt, sl = cache.page_table, cache.seq_lens
-    assert pt.dtype == torch.int32 and sl.dtype == torch.int32 and pt.is_contiguous()
+    if k.dtype != torch.bfloat16 or v.dtype != torch.bfloat16:
+        raise ValueError("KV cache: k and v must be bf16, got %s / %s" % (k.dtype, v.dtype))
+    if k.dim() != 4 or k.shape != v.shape or not k.is_contiguous() or not v.is_contiguous():
+        raise ValueError("KV cache: k and v must be contiguous [num_pages][Hkv][P][d] tensors of one shape")
+    if pt.dtype != torch.int32 or pt.dim() != 2 or not pt.is_contiguous():
+        raise ValueError("KV cache: page_table must be a contiguous int32 [B][max_pages] tensor")
+    if sl.dtype != torch.int32 or tuple(sl.shape) != (pt.shape[0],) or not sl.is_contiguous():
+        raise ValueError("KV cache: seq_lens must be a contiguous int32 [B] tensor, B = %d" % pt.shape[0])
+    devs = {t.device for t in (k, v, pt, sl)}
+    if device is not None:
+        devs.add(torch.device(device))
+    if len(devs) != 1:
+        raise ValueError("KV cache: k, v, page_table, seq_lens and the queries must be on one device, got %s"
+                         % sorted(str(d) for d in devs))
     return L.KVCacheS(k.data_ptr(), v.data_ptr(), pt.data_ptr(), sl.data_ptr(), pt.shape[0], k.shape[1],
                       k.shape[3], k.shape[2], pt.shape[1], k.shape[0])
 
 
 class Workspace:
-    """A reusable, zero-initialised device workspace (grows on demand)."""
+    """A reusable, zero-initialised device workspace (grows on demand).
+
+    A workspace belongs to one stream at a time: calls that share it must be
+    ordered on the GPU (same stream, or events between streams), since every
+    call rewrites its status header and scratch.  When it grows, the old
+    buffer is released with record_stream() for every stream it was handed
+    to, so the caching allocator does not reuse that memory while a kernel
+    launched on one of those streams may still read it."""
 
     def __init__(self, device=None):
         self.device = device
         self.buf: Optional[torch.Tensor] = None
+        self._streams = []
 
-    def get(self, nbytes: int) -> torch.Tensor:
+    def get(self, nbytes: int, stream=None) -> torch.Tensor:
         if self.buf is None or self.buf.numel() < nbytes:
             n = max(nbytes, 256)
+            old = self.buf
             self.buf = torch.zeros(n + 256, dtype=torch.uint8, device=self.device or "cuda")
+            if old is not None:
+                for s in self._streams:
+                    old.record_stream(s)
+            self._streams = []
+        if self.buf.device.type == "cuda":
+            s = stream if stream is not None else torch.cuda.current_stream(self.buf.device)
+            if all(s != x for x in self._streams):
+                self._streams.append(s)
         return self.buf
 
-    def aligned(self, nbytes: int):
-        buf = self.get(nbytes)
+    def aligned(self, nbytes: int, stream=None):
+        buf = self.get(nbytes, stream)
         base = buf.data_ptr()
         off = (-base) % 256
         return ctypes.c_void_p(base + off), buf.numel() - off
@@ -95,7 +124,7 @@ class Workspace:
         """Synchronise and return (status, detail) recorded by kernels (then cleared)."""
         if self.buf is None:
             return 0, (0, 0, 0)
-        ptr, _ = self.aligned(0)
+        ptr, _ = self.aligned(0, stream)
         det = (L.c_i32 * 3)()
         st = L.load().sa_read_device_status(ptr, _stream(stream), det)
         return st, tuple(det)
@@ -109,10 +138,19 @@ class Workspace:
 _default_ws = {}
 
 
-def _ws(ws: Optional[Workspace], device) -> Workspace:
+def _ws(ws: Optional[Workspace], device, stream=None) -> Workspace:
+    """The caller's workspace, else a default one per (device, stream), so
+    that calls on different streams never share scratch."""
     if ws is not None:
         return ws
-    key = str(device)
+    dev = torch.device(device)
+    if stream is not None:
+        sid = int(stream.cuda_stream)
+    elif dev.type == "cuda":
+        sid = int(torch.cuda.current_stream(dev).cuda_stream)
+    else:
+        sid = 0
+    key = (str(dev), sid)
     if key not in _default_ws:
         _default_ws[key] = Workspace(device)
     return _default_ws[key]
@@ -183,6 +221,26 @@ class BlockCSR:
     num_q_blocks: int
 
 
+def _check_selection(sel, B: int, Hq: int, device) -> None:
+    """The selection tensors a decode reads must have the layout the kernels
+    index: token lists idx int32 [B][Hq][k_cap] and count int32 [B][Hq];
+    block lists blocks int32 [B][max_blocks][4] and block_counts int32 [B];
+    contiguous, on the queries' device.  Raises ValueError otherwise."""
+    if isinstance(sel, TokenSelection):
+        if sel.idx.dim() != 3:
+            raise ValueError("TokenSelection.idx must be int32 [B][Hq][k_cap], got shape %s" % (tuple(sel.idx.shape),))
+        _need(sel.idx, (B, Hq, sel.idx.shape[-1]), torch.int32, device, "TokenSelection.idx")
+        _need(sel.count, (B, Hq), torch.int32, device, "TokenSelection.count")
+    elif isinstance(sel, BlockSelection):
+        if sel.blocks.dim() != 3:
+            raise ValueError("BlockSelection.blocks must be int32 [B][max_blocks][4], got shape %s"
+                             % (tuple(sel.blocks.shape),))
+        _need(sel.blocks, (B, sel.blocks.shape[1], 4), torch.int32, device, "BlockSelection.blocks")
+        _need(sel.block_counts, (B,), torch.int32, device, "BlockSelection.block_counts")
+    else:
+        raise TypeError("selection must be a TokenSelection or a BlockSelection, got %s" % type(sel).__name__)
+
+
 # --------------------------------------------------------------------------
 # entry points
 # --------------------------------------------------------------------------
@@ -199,9 +257,9 @@ def select_topk(cache, q: torch.Tensor, k: int, idx: Optional[torch.Tensor] = No
     if count is None:
         count = torch.empty((B, Hq), dtype=torch.int32, device=dev)
     _need(count, (B, Hq), torch.int32, dev, "select_topk count")
-    kv = kv_struct(cache)
-    w = _ws(ws, dev)
-    wp, wn = w.aligned(workspace_bytes(L.OP_SELECT_TOPK, cache, num_q_heads=Hq, k=k))
+    kv = kv_struct(cache, dev)
+    w = _ws(ws, dev, stream)
+    wp, wn = w.aligned(workspace_bytes(L.OP_SELECT_TOPK, cache, num_q_heads=Hq, k=k), stream)
     _check(L.load().sa_select_topk(ctypes.byref(kv), _ptr(q.contiguous()), _qdtype(q), Hq, k, _ptr(idx),
                                    _ptr(count), wp, wn, _stream(stream)), "sa_select_topk")
     return TokenSelection(idx, count)
@@ -222,10 +280,11 @@ def sparse_decode_attn(cache, q: torch.Tensor, sel, scale: Optional[float] = Non
         lse = torch.empty((B, Hq), dtype=torch.float32, device=dev)
     if lse is not None:
         _need(lse, (B, Hq), torch.float32, dev, "sparse_decode_attn lse")
-    kv = kv_struct(cache)
+    kv = kv_struct(cache, dev)
+    _check_selection(sel, B, Hq, dev)
     s = sel.struct()
-    w = _ws(ws, dev)
-    wp, wn = w.aligned(workspace_bytes(L.OP_DECODE, cache, num_q_heads=Hq, num_splits=num_splits))
+    w = _ws(ws, dev, stream)
+    wp, wn = w.aligned(workspace_bytes(L.OP_DECODE, cache, num_q_heads=Hq, num_splits=num_splits), stream)
     _check(L.load().sa_sparse_decode_attn(ctypes.byref(kv), _ptr(q.contiguous()), _qdtype(q), Hq,
                                           ctypes.byref(s), scale, num_splits, _ptr(out), _ptr(lse), wp, wn,
                                           _stream(stream)), "sa_sparse_decode_attn")
@@ -248,8 +307,8 @@ def fetch_pages(host_k: torch.Tensor, host_v: torch.Tensor, dev_k: torch.Tensor,
     if pairs.dtype != torch.int32 or pairs.dim() != 2 or pairs.shape[1] != 2 or not pairs.is_contiguous():
         raise ValueError("pairs must be a contiguous int32 [n][2] tensor")
     page_bytes = host_k[0].numel() * 2 if host_k.shape[0] else dev_k[0].numel() * 2
-    w = _ws(ws, dev_k.device)
-    wp, wn = w.aligned(256)
+    w = _ws(ws, dev_k.device, stream)
+    wp, wn = w.aligned(256, stream)
     _check(L.load().sa_fetch_pages(host_k.data_ptr(), host_v.data_ptr(), dev_k.data_ptr(), dev_v.data_ptr(),
                                    pairs.data_ptr(), pairs.shape[0], host_k.shape[0], dev_k.shape[0], page_bytes,
                                    wp, wn, _stream(stream)), "sa_fetch_pages")
@@ -275,15 +334,15 @@ def select_blocks_spans(cache, spans: torch.Tensor, span_counts: torch.Tensor, s
     if span_round.dtype == torch.bool:
         span_round = span_round.to(torch.uint8)
     _need(span_round, (B, S), torch.uint8, dev, "select_blocks_spans span_round")
-    kv = kv_struct(cache)
+    kv = kv_struct(cache, dev)
     a = L.BlockSelectArgsS()
     a.mode = L.SEL_SPANS
     a.spans, a.span_counts, a.span_round = spans.data_ptr(), span_counts.data_ptr(), span_round.data_ptr()
     a.max_spans = spans.shape[1]
     o = L.BlockListS()
     o.blocks, o.block_counts, o.max_blocks = out.blocks.data_ptr(), out.block_counts.data_ptr(), out.blocks.shape[1]
-    w = _ws(ws, dev)
-    wp, wn = w.aligned(workspace_bytes(L.OP_SELECT_BLOCKS, cache, block_args=a))
+    w = _ws(ws, dev, stream)
+    wp, wn = w.aligned(workspace_bytes(L.OP_SELECT_BLOCKS, cache, block_args=a), stream)
     _check(L.load().sa_select_blocks(ctypes.byref(kv), ctypes.byref(a), ctypes.byref(o), wp, wn,
                                      _stream(stream)), "sa_select_blocks(spans)")
     return out
@@ -315,7 +374,7 @@ def select_blocks_rbs(cache, q: torch.Tensor, block_size: int = 64, scale: Optio
     if tau_c is not None:
         tc = torch.as_tensor(tau_c, dtype=torch.float32, device=dev).expand(Hq).contiguous()
         tr = torch.as_tensor(tau_r, dtype=torch.float32, device=dev).expand(Hq).contiguous()
-    kv = kv_struct(cache)
+    kv = kv_struct(cache, dev)
     a = L.BlockSelectArgsS()
     a.mode = L.SEL_RBS
     a.q = q.data_ptr()
@@ -327,8 +386,8 @@ def select_blocks_rbs(cache, q: torch.Tensor, block_size: int = 64, scale: Optio
     o = L.BlockListS()
     o.row_ptr, o.cols, o.nnz_capacity = out.row_ptr.data_ptr(), out.cols.data_ptr(), out.cols.numel()
     o.tau_out = out.tau.data_ptr()
-    w = _ws(ws, dev)
-    wp, wn = w.aligned(workspace_bytes(L.OP_SELECT_BLOCKS, cache, block_args=a))
+    w = _ws(ws, dev, stream)
+    wp, wn = w.aligned(workspace_bytes(L.OP_SELECT_BLOCKS, cache, block_args=a), stream)
     _check(L.load().sa_select_blocks(ctypes.byref(kv), ctypes.byref(a), ctypes.byref(o), wp, wn,
                                      _stream(stream)), "sa_select_blocks(rbs)")
     return out
@@ -353,11 +412,11 @@ def sparse_prefill_attn(cache, q: torch.Tensor, csr: BlockCSR, scale: Optional[f
     nQB = (T + 63) // 64
     _need(csr.row_ptr, (Hq * nQB + 1,), torch.int32, dev, "sparse_prefill_attn csr.row_ptr")
     _need(csr.cols, (csr.cols.numel(),), torch.int32, dev, "sparse_prefill_attn csr.cols")
-    kv = kv_struct(cache)
+    kv = kv_struct(cache, dev)
     c = L.BlockListS()
     c.row_ptr, c.cols, c.nnz_capacity = csr.row_ptr.data_ptr(), csr.cols.data_ptr(), csr.cols.numel()
-    w = _ws(ws, dev)
-    wp, wn = w.aligned(workspace_bytes(L.OP_PREFILL, cache, num_q_heads=Hq, num_tokens=T))
+    w = _ws(ws, dev, stream)
+    wp, wn = w.aligned(workspace_bytes(L.OP_PREFILL, cache, num_q_heads=Hq, num_tokens=T), stream)
     _check(L.load().sa_sparse_prefill_attn(ctypes.byref(kv), _ptr(q), Hq, T, ctypes.byref(c), scale, 1,
                                            _ptr(out), _ptr(lse), wp, wn, _stream(stream)),
            "sa_sparse_prefill_attn")

@@ -10,6 +10,17 @@
 
 using namespace sa;
 
+namespace sa {
+// status header + split-KV partial outputs + (m, l) pairs, each rounded up to
+// 256 bytes (the layout sa_sparse_decode_attn carves out of its workspace)
+size_t decode_workspace_bytes(const sa_kv_cache *kv, int Hq, int S)
+{
+    const size_t rows = (size_t)kv->batch * Hq;
+    auto up = [](size_t x) { return (x + 255) / 256 * 256; };
+    return sizeof(DevStatus) + up(rows * S * kv->head_dim * sizeof(float)) + up(rows * S * 2 * sizeof(float));
+}
+}  // namespace sa
+
 namespace {
 
 constexpr size_t kAlign = 256;
@@ -80,11 +91,7 @@ size_t ws_topk(const sa_kv_cache *kv, int Hq)
     return kHeader + up((size_t)kv->batch * Hq * Lcap * sizeof(float));
 }
 
-size_t ws_decode(const sa_kv_cache *kv, int Hq, int S)
-{
-    const size_t rows = (size_t)kv->batch * Hq;
-    return kHeader + up(rows * S * kv->head_dim * sizeof(float)) + up(rows * S * 2 * sizeof(float));
-}
+size_t ws_decode(const sa_kv_cache *kv, int Hq, int S) { return sa::decode_workspace_bytes(kv, Hq, S); }
 
 size_t ws_blocks(const sa_kv_cache *kv, const sa_block_select_args *a)
 {

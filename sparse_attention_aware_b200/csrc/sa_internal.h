@@ -40,6 +40,8 @@ struct DecodeArgs {
     DevStatus *st;
 };
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+// bytes of workspace sa_sparse_decode_attn needs (status header + partials)
+size_t decode_workspace_bytes(const sa_kv_cache *kv, int Hq, int S);
 
 // ---- host-tier page fetch ---------------------------------------------------
 struct FetchArgs {

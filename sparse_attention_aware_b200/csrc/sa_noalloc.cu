@@ -18,7 +18,6 @@ using namespace sa;
 namespace {
 
 constexpr size_t kNoAllocBytes = SA_NOALLOC_DECODE_SCRATCH_BYTES;
-constexpr size_t kHead = 256;   // status header, as in a workspace
 constexpr int kMaxDevices = 128;
 
 // Every GPU that loads libsa holds this array until the process exits.
@@ -49,8 +48,6 @@ sa_status scratch_address(void **out)
     return SA_OK;
 }
 
-inline size_t round_up(size_t x) { return (x + 255) / 256 * 256; }
-
 }  // namespace
 
 extern "C" sa_status sa_sparse_decode_attn_noalloc(const sa_kv_cache *kv, const void *q, sa_dtype q_dtype,
@@ -67,10 +64,9 @@ extern "C" sa_status sa_sparse_decode_attn_noalloc(const sa_kv_cache *kv, const 
     if (kv->page_size != 16 && kv->page_size != 64) return SA_ERR_UNSUPPORTED;
     if (num_q_heads <= 0 || num_splits < 1 || num_splits > 64) return SA_ERR_INVALID_ARGUMENT;
     if (num_q_heads % kv->num_kv_heads) return SA_ERR_UNSUPPORTED;
-    const size_t rows = (size_t)kv->batch * num_q_heads;
-    const size_t need = kHead + round_up(rows * num_splits * kv->head_dim * sizeof(float)) +
-                        round_up(rows * num_splits * 2 * sizeof(float));
-    if (need > kNoAllocBytes) return SA_ERR_UNSUPPORTED;   // beyond the built-in scratch
+    // the same layout the workspace entry point carves out of its workspace
+    if (decode_workspace_bytes(kv, num_q_heads, num_splits) > kNoAllocBytes)
+        return SA_ERR_UNSUPPORTED;   // beyond the built-in scratch
     void *base = nullptr;
     sa_status st = scratch_address(&base);
     if (st != SA_OK) return st;

@@ -167,6 +167,41 @@ def test_bench_prefill_config(cuda_dev):
     np.testing.assert_allclose(lse.cpu().numpy().reshape(-1)[rows], ref_lse, atol=2e-3, rtol=0)
 
 
+def test_bench_prefill_config_at_bench_density(cuda_dev):
+    """The prefill exactly as the bench times it: 131072 tokens, 32/4 heads,
+    the bench's quantile levels (p_c = 0.9648, p_r = p_c + 0.02, ~5% kept
+    blocks including the forced ones), per-head thresholds read back from the
+    quantile-mode call and passed explicitly, and the CSR that selection
+    produced executed by the tcgen05 kernel.  The oracle attends over the mask
+    read back from that CSR (mask bit-exactness is the gap-threshold test's
+    job) on 260 sampled rows, the first and last query blocks included."""
+    wl = W.clustered_prefill(1005, device=cuda_dev, T=131072, Hq=32, Hkv=4, d=128, block=64)
+    T, Hq, d = wl.q.shape
+    nB = T // 64
+    scale = 1 / math.sqrt(128)
+    ws = sa.Workspace(cuda_dev)
+    pc = 0.9648
+    q_csr = sa.select_blocks_rbs(wl.cache, wl.q, 64, scale, p_c=pc, p_r=pc + 0.02, ws=ws)
+    ws.raise_on_fault()
+    tau = q_csr.tau.clone()
+    csr = sa.select_blocks_rbs(wl.cache, wl.q, 64, scale, tau_c=tau[0], tau_r=tau[1], ws=ws)
+    ws.raise_on_fault()
+    mask = csr_to_mask(csr.row_ptr.cpu().numpy(), csr.cols.cpu().numpy(), Hq, nB)
+    assert 0.045 <= mask.mean() <= 0.055, mask.mean()
+    out, lse = sa.sparse_prefill_attn(wl.cache, wl.q, csr, scale, ws=ws)
+    ws.raise_on_fault()
+    rng = np.random.default_rng(29)
+    ts = np.concatenate([[0, 1, 63, 64, 127, T - 64, T - 63, T - 2, T - 1],
+                         rng.integers(0, 64, 8), rng.integers(T - 64, T, 8), rng.integers(0, T, 235)])
+    hs = rng.integers(0, Hq, len(ts))
+    rows = (ts * Hq + hs).astype(np.int64)
+    cpu = wl.cache.to("cpu")
+    ref, ref_lse = oracle.prefill(cpu, wl.q.cpu(), 64, mask, scale, rows=rows)
+    g_out = out.float().cpu().numpy().reshape(-1, d)[rows]
+    assert_close_attn(g_out, ref)
+    np.testing.assert_allclose(lse.cpu().numpy().reshape(-1)[rows], ref_lse, atol=2e-3, rtol=0)
+
+
 def _schedule_items(ws, Hq, Hkv, nB):
     """Work items the last prefill call left in its workspace (after the
     256-byte status header): {head A, block A, head B (-1: none), block B}."""

@@ -19,7 +19,7 @@ def _cache():
 def test_workspace_allocation_failure_propagates(monkeypatch):
     cache, q = _cache()
 
-    def fail(self, nbytes):
+    def fail(self, nbytes, stream=None):
         raise MemoryError("injected: device workspace allocation failed")
 
     monkeypatch.setattr(api.Workspace, "get", fail)
@@ -74,3 +74,43 @@ def test_caller_tensors_with_the_wrong_layout_are_rejected_before_launch():
         sa.sparse_prefill_attn(wl.cache, wl.q, sa.BlockCSR(torch.zeros(5, dtype=torch.int32), csr.cols, csr.tau, 2, 4))
     with pytest.raises(ValueError, match="sparse_prefill_attn out"):
         sa.sparse_prefill_attn(wl.cache, wl.q, csr, out=torch.zeros((200, 2, 128), dtype=torch.bfloat16)[:, :1])
+
+
+def test_selection_tensors_with_the_wrong_layout_are_rejected_before_launch():
+    """The decode reads the selection tensors by the (B, Hq) shape of its
+    queries: a short count, a wide index type, a non-contiguous index or a
+    block list of the wrong width must raise before anything is launched."""
+    cache, q = _cache()                       # B=1, Hq=4
+    idx = torch.zeros((1, 4, 8), dtype=torch.int32)
+    cnt = torch.zeros((1, 4), dtype=torch.int32)
+    bad = [
+        (sa.TokenSelection(idx, torch.zeros((1, 3), dtype=torch.int32)), "TokenSelection.count"),
+        (sa.TokenSelection(idx.long(), cnt), "TokenSelection.idx"),
+        (sa.TokenSelection(torch.zeros((1, 8, 4), dtype=torch.int32).transpose(1, 2), cnt), "TokenSelection.idx"),
+        (sa.TokenSelection(torch.zeros((2, 4, 8), dtype=torch.int32), cnt), "TokenSelection.idx"),
+        (sa.BlockSelection(torch.zeros((1, 5, 3), dtype=torch.int32), torch.zeros((1,), dtype=torch.int32)),
+         "BlockSelection.blocks"),
+        (sa.BlockSelection(torch.zeros((1, 5, 4), dtype=torch.int32), torch.zeros((2,), dtype=torch.int32)),
+         "BlockSelection.block_counts"),
+    ]
+    for sel, what in bad:
+        with pytest.raises(ValueError, match=what):
+            sa.sparse_decode_attn(cache, q, sel, 0.1, 2)
+    with pytest.raises(TypeError, match="TokenSelection or a BlockSelection"):
+        sa.sparse_decode_attn(cache, q, (idx, cnt), 0.1, 2)
+
+
+def test_cache_descriptors_are_checked_without_asserts():
+    """kv_struct raises ValueError (not assert, which python -O drops) for a
+    short seq_lens, a wrong dtype, or cache tensors on another device."""
+    import dataclasses
+    cache, q = _cache()
+    short = dataclasses.replace(cache, seq_lens=torch.zeros((0,), dtype=torch.int32))
+    with pytest.raises(ValueError, match="seq_lens"):
+        api.kv_struct(short)
+    with pytest.raises(ValueError, match="bf16"):
+        api.kv_struct(dataclasses.replace(cache, k=cache.k.float()))
+    with pytest.raises(ValueError, match="page_table"):
+        api.kv_struct(dataclasses.replace(cache, page_table=cache.page_table.long()))
+    with pytest.raises(ValueError, match="one device"):
+        api.kv_struct(cache, torch.device("meta"))
