@@ -46,12 +46,11 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 
 # kernels each API call launches (libsa): top-k = score + select; decode =
 # split + combine; spans = 1; RBS with explicit thresholds = block statistics,
-# query pooling, pair tiles, 3 CSR scan kernels, CSR fill; prefill = schedule +
-# tcgen05 kernel
+# query pooling, pair tiles, CSR fill; prefill = schedule + tcgen05 kernel
 # splits of the masked-decode step (a sequence uses only as many as give each
 # ~128 tokens; 16 measured best on the 131072-token step: 34.1 vs 35.9 us at 8)
 MASKED_SPLITS = 16
-LAUNCHES = {"select_topk": 2, "decode": 2, "spans": 1, "rbs_explicit": 7, "prefill": 2}
+LAUNCHES = {"select_topk": 2, "decode": 2, "spans": 1, "rbs_explicit": 4, "prefill": 2}
 
 
 def pct(xs, q):
@@ -532,6 +531,7 @@ def tiered_measure(msk, cfg, dev, steps=64, slot_frac=0.125):
     machines = [DA.DAStateMachine(L - steps) for _ in range(m["B"])]
     ws = sa.Workspace(dev)
     out = torch.empty((m["B"], m["Hq"], m["d"]), dtype=torch.bfloat16, device=dev)
+    packer = SP.SpanPacker(m["B"], 2, dev)
 
     def tokens(i, b):
         # per 16 steps: <local>, a focus declaration on chunks (c0, c0 + 1)
@@ -549,7 +549,7 @@ def tiered_measure(msk, cfg, dev, steps=64, slot_frac=0.125):
         for b, mach in enumerate(machines):
             mach.observe(tokens(i, b))
             lists.append(mach.next_spans(lens[b]))
-        spans, cnt, rnd = SP.pack(lists, dev, max_spans=2)
+        spans, cnt, rnd = packer.pack(lists)
         tier.prepare([T.span_pages(l, n, P) for l, n in zip(lists, lens)], seq_lens=lens)
         c = tier.cache
         sel = sa.select_blocks_spans(c, spans, cnt, rnd, ws=ws)
