@@ -8,7 +8,8 @@ workload generators.  Build the library with
 from .api import (BlockCSR, BlockSelection, SAError, TokenSelection, Workspace, fetch_pages, select_blocks_rbs,
                   select_blocks_spans, select_topk, sparse_decode_attn, sparse_prefill_attn,
                   workspace_bytes)
+from .cache import PagedCache
 
 __all__ = ["select_topk", "select_blocks_rbs", "select_blocks_spans", "sparse_decode_attn",
            "sparse_prefill_attn", "workspace_bytes", "Workspace", "TokenSelection", "BlockSelection",
-           "BlockCSR", "SAError", "fetch_pages"]
+           "BlockCSR", "SAError", "fetch_pages", "PagedCache"]

@@ -60,3 +60,57 @@ def pack(span_lists: Sequence[Sequence[Tuple[int, int, bool]]], device="cuda", m
             rnd[b, :n] = [1 if r else 0 for _, _, r in lst]
     return (torch.from_numpy(spans).to(device), torch.from_numpy(cnt).to(device),
             torch.from_numpy(rnd).to(device))
+
+
+class SpanPacker:
+    """``pack`` for a serving loop: the span lists of a step are written into
+    one of ``depth`` pinned host buffers and copied to fixed device tensors
+    with non-blocking copies on the caller's stream, so the host does not wait
+    for the GPU (a copy from pageable memory would wait for the stream).  A
+    host buffer is rewritten only after the copy that last read it has
+    completed; the device tensors are rewritten by a copy queued on the same
+    stream as the kernels that read them, so stream order protects them."""
+
+    def __init__(self, batch: int, max_spans: int, device, depth: int = 2):
+        import numpy as np
+        self.B, self.S = batch, max(1, max_spans)
+        self.device = torch.device(device)
+        self.host = [(torch.zeros((batch, self.S, 2), dtype=torch.int32).pin_memory(),
+                      torch.zeros((batch,), dtype=torch.int32).pin_memory(),
+                      torch.zeros((batch, self.S), dtype=torch.uint8).pin_memory()) for _ in range(depth)]
+        self.done = [None] * depth
+        self.dev = (torch.zeros((batch, self.S, 2), dtype=torch.int32, device=self.device),
+                    torch.zeros((batch,), dtype=torch.int32, device=self.device),
+                    torch.zeros((batch, self.S), dtype=torch.uint8, device=self.device))
+        self.i = 0
+        self._np = np
+
+    def pack(self, span_lists: Sequence[Sequence[Tuple[int, int, bool]]], stream=None):
+        """Device (spans, counts, round) for ``span_lists`` (one list per
+        sequence, at most ``max_spans`` spans each)."""
+        if len(span_lists) != self.B:
+            raise ValueError("need one span list per sequence (%d)" % self.B)
+        k = self.i % len(self.host)
+        self.i += 1
+        if self.done[k] is not None:
+            self.done[k].synchronize()
+        hs, hc, hr = self.host[k]
+        ns, nc, nr = hs.numpy(), hc.numpy(), hr.numpy()
+        ns[...] = 0
+        nc[...] = 0
+        nr[...] = 0
+        for b, lst in enumerate(span_lists):
+            n = len(lst)
+            if n > self.S:
+                raise ValueError("sequence %d has %d spans, the packer holds %d" % (b, n, self.S))
+            nc[b] = n
+            for j, (s0, s1, r) in enumerate(lst):
+                ns[b, j, 0], ns[b, j, 1], nr[b, j] = s0, s1, 1 if r else 0
+        s = stream if stream is not None else torch.cuda.current_stream(self.device)
+        with torch.cuda.stream(s):
+            for d, h in zip(self.dev, self.host[k]):
+                d.copy_(h, non_blocking=True)
+            ev = torch.cuda.Event()
+            ev.record(s)
+        self.done[k] = ev
+        return self.dev

@@ -26,7 +26,7 @@ import numpy as np
 import torch
 
 from . import api
-from .workloads import PagedCache
+from .cache import PagedCache
 
 
 def span_pages(spans: Sequence[Tuple[int, int, bool]], seq_len: int, page_size: int) -> List[int]:

@@ -25,6 +25,8 @@ from typing import List, Optional, Sequence
 
 import torch
 
+from .cache import PagedCache  # noqa: F401  (re-exported: generators build caches)
+
 # stream ids
 S_Q, S_K, S_V, S_STRUCT, S_PERM, S_MODES, S_REDRAW, S_OUTLIER, S_PAD = range(1, 10)
 
@@ -61,45 +63,6 @@ def randn(shape, seed, stream, sub=0, device="cpu", dtype=torch.float32):
 # --------------------------------------------------------------------------
 # paged cache
 # --------------------------------------------------------------------------
-@dataclasses.dataclass
-class PagedCache:
-    k: torch.Tensor            # bf16 [num_pages][Hkv][P][d]
-    v: torch.Tensor            # bf16 [num_pages][Hkv][P][d]
-    page_table: torch.Tensor   # int32 [B][max_pages]
-    seq_lens: torch.Tensor     # int32 [B]
-
-    @property
-    def batch(self) -> int:
-        return int(self.page_table.shape[0])
-
-    @property
-    def num_kv_heads(self) -> int:
-        return int(self.k.shape[1])
-
-    @property
-    def page_size(self) -> int:
-        return int(self.k.shape[2])
-
-    @property
-    def head_dim(self) -> int:
-        return int(self.k.shape[3])
-
-    @property
-    def max_pages(self) -> int:
-        return int(self.page_table.shape[1])
-
-    @property
-    def num_pages(self) -> int:
-        return int(self.k.shape[0])
-
-    def with_v(self, v: torch.Tensor) -> "PagedCache":
-        return PagedCache(self.k, v, self.page_table, self.seq_lens)
-
-    def to(self, device) -> "PagedCache":
-        return PagedCache(self.k.to(device), self.v.to(device),
-                          self.page_table.to(device), self.seq_lens.to(device))
-
-
 def page_permutation(num_pages: int, seed: int, shuffle: bool, device="cpu") -> torch.Tensor:
     if not shuffle:
         return torch.arange(num_pages, dtype=torch.int64, device=device)

@@ -261,3 +261,30 @@ def test_da_state_machine_drives_masked_decode(cuda_dev):
         assert_close_attn(out.float().cpu().numpy().reshape(-1, d), ref)
         np.testing.assert_allclose(lse.cpu().numpy().reshape(-1), ref_lse, atol=2e-3, rtol=0)
     ws.raise_on_fault()
+
+
+def test_span_packer_matches_pack_over_steps(cuda_dev):
+    """The non-blocking packer gives the same device tensors as pack() for a
+    run of steps, with its pinned buffers reused (depth 2) and the previous
+    step's selection still queued when the next step is packed."""
+    rng = np.random.default_rng(5)
+    cache, _ = W.random_decode(9, 3, 2, 1, 64, [3000, 4096, 777], 16)
+    gc = cache.to(cuda_dev)
+    packer = SP.SpanPacker(3, 2, cuda_dev)
+    ws = sa.Workspace(cuda_dev)
+    for step in range(6):
+        lists = []
+        for L in (3000, 4096, 777):
+            n = int(rng.integers(0, 3))
+            lists.append([(int(a), int(a) + int(rng.integers(1, 900)), bool(rng.integers(0, 2)))
+                          for a in rng.integers(-20, L, n)])
+        want = SP.pack(lists, cuda_dev, max_spans=2)
+        got = packer.pack(lists)
+        sel_w = sa.select_blocks_spans(gc, *want, ws=ws)
+        sel_g = sa.select_blocks_spans(gc, *got, ws=ws)
+        torch.cuda.synchronize()
+        for x, y in zip(got, want):
+            assert torch.equal(x, y)
+        assert torch.equal(sel_g.block_counts, sel_w.block_counts)
+        n = sel_w.block_counts.max().item()
+        assert torch.equal(sel_g.blocks[:, :n], sel_w.blocks[:, :n])
