@@ -297,11 +297,7 @@ __global__ void __launch_bounds__(kThr, 1) k_pair_tc(const RbsArgs a, int nTB)
             fence_before_sync();
             mbar_arrive(acc_free + s);
         }
-        if (!QUANT) {
-            if (row_ok && kept) atomicAdd(&a.rowcnt[h * a.nB + i], kept);
-            const int wk = warp_sum(row_ok ? kept : 0);   // this warp's rows and column half
-            if (lane == 0 && wk) atomicAdd(&a.tilecnt[(size_t)h * nTB + I], wk);
-        }
+        if (!QUANT && row_ok && kept) atomicAdd(&a.rowcnt[h * a.nB + i], kept);
     }
 
     __syncthreads();

@@ -22,8 +22,7 @@
 //   k_qhist/k_qpick  find each head's lower quantile (exact radix select on
 //                  the order-preserving key, grid-wide histograms) and
 //   k_mask_scores  thresholds the stored scores.
-//   k_csr_fill     turns counts and bits into CSR (ascending cols), one CTA per
-//                  128-row tile placed by the tile totals before it.
+//   k_csr_scan / k_csr_fill  turn counts and bits into CSR (ascending cols).
 #include <cuda_bf16.h>
 
 #include "sa_internal.h"
@@ -43,7 +42,7 @@ size_t rbs_workspace_layout(int Hq, int Hkv, int D, int nB, bool quantile, size_
     offs[3] = o; o += up((size_t)Hq * nB * 4);            // pooled query norms
     offs[4] = o; o += up((size_t)2 * Hq * 4);             // thresholds
     offs[5] = o; o += up((size_t)Hq * nB * words * 4);    // mask bits
-    offs[6] = o; o += up((size_t)Hq * nB * 4 + (size_t)Hq * rbs_img_tiles(nB) * 4 + 16);   // row counts + tile totals
+    offs[6] = o; o += up((size_t)Hq * nB * 4 + 16 + ((size_t)Hq * nB / 1024 + 2) * 8);   // row counts + chunk sums
     offs[7] = o; if (quantile) o += up((size_t)2 * Hq * nP * 4);   // pair scores
     // radix-select scratch: per (branch, head) a 2048-bin histogram for each of
     // the 3 digit passes + state {prefix, mask, need}
@@ -180,10 +179,7 @@ __device__ void pool_q_cta(const RbsArgs &a, PoolSmem &sm, int i, int h)
         }
         return;
     }
-    if (threadIdx.x == 0) {
-        a.rowcnt[(size_t)h * a.nB + i] = 0;
-        if ((i & (kRbsImgRows - 1)) == 0) a.tilecnt[(size_t)h * rbs_img_tiles(a.nB) + (i >> 7)] = 0;
-    }
+    if (threadIdx.x == 0) a.rowcnt[(size_t)h * a.nB + i] = 0;
     const int n = min(BS, a.T - i * BS);
     const int lane16 = threadIdx.x & 15, rs = threadIdx.x >> 4;   // 16 row slots
     float acc[8] = {0, 0, 0, 0, 0, 0, 0, 0};
@@ -225,17 +221,12 @@ __global__ void __launch_bounds__(256) k_block_stats(const RbsArgs a)
     block_stats_cta(a, *reinterpret_cast<StatsSmem *>(raw), blockIdx.x, blockIdx.y);
 }
 
-// Pooling reads only the queries and writes nothing the statistics kernel
-// before it reads, so it does not wait for that kernel to finish before
-// starting: it is launched once the statistics kernel has started (which has
-// itself waited for the work before it), runs alongside it, and waits for it
-// only before exiting, so that the pair kernel after it sees both.
 __global__ void __launch_bounds__(256) k_pool_q(const RbsArgs a)
 {
+    pdl_wait();
     pdl_trigger();
     __shared__ __align__(16) uint8_t raw[sizeof(PoolSmem)];
     pool_q_cta(a, *reinterpret_cast<PoolSmem *>(raw), blockIdx.x, blockIdx.y);
-    pdl_wait();
 }
 
 // ---------------------------------------------------------------------------
@@ -409,76 +400,91 @@ __global__ void __launch_bounds__(256) k_mask_scores(const RbsArgs a)
             cnt += __popc(w);
         }
     }
-    if (lane == 0) {
-        a.rowcnt[row] = cnt;
-        if (cnt) atomicAdd(&a.tilecnt[(size_t)h * rbs_img_tiles(a.nB) + (i >> 7)], cnt);
-    }
+    if (lane == 0) a.rowcnt[row] = cnt;
 }
 
-// CSR, one CTA per (head, 128-row tile) in row order: the tile's first entry
-// is the sum of the kept counts of the tiles before it (tile totals, summed by
-// whichever kernel produced the row counts), the rows' pointers follow by an
-// exclusive scan of their counts, and one warp per row writes its columns
-// in ascending order.
-__global__ void __launch_bounds__(256) k_csr_fill(const RbsArgs a, int nTB)
+// CSR row pointers: exclusive prefix sum of the row counts in three short
+// launches (per-chunk sums, one scan of the chunk sums, per-chunk write-out).
+constexpr int kScanChunk = 1024;   // rows per CTA (one per thread)
+
+__global__ void __launch_bounds__(kScanChunk) k_csr_sum(const RbsArgs a, long long *chunk_sum)
 {
     pdl_wait();
     pdl_trigger();
     __shared__ long long wt[33];
-    __shared__ long long s_base[kRbsImgRows];
-    const int tile = blockIdx.x;                 // h * nTB + I
-    const int h = tile / nTB, I = tile % nTB;
+    const int R = a.Hq * a.nB;
+    const int r = blockIdx.x * kScanChunk + threadIdx.x;
+    long long total;
+    block_excl_scan_ll(r < R ? a.rowcnt[r] : 0, wt, total);
+    if (threadIdx.x == 0) chunk_sum[blockIdx.x] = total;
+}
+
+__global__ void __launch_bounds__(1024) k_csr_chunks(const RbsArgs a, long long *chunk_sum, int nchunks)
+{
+    pdl_wait();
+    pdl_trigger();
+    __shared__ long long wt[33];
+    long long run = 0;
+    for (int c0 = 0; c0 < nchunks; c0 += 1024) {
+        const int c = c0 + threadIdx.x;
+        const long long v = c < nchunks ? chunk_sum[c] : 0;
+        long long total;
+        const long long ex = block_excl_scan_ll(v, wt, total);
+        if (c < nchunks) chunk_sum[c] = run + ex;
+        run += total;
+    }
+    if (threadIdx.x == 0) {
+        const int R = a.Hq * a.nB;
+        a.row_ptr[R] = (int32_t)min(run, (long long)INT32_MAX);
+        if (run > a.nnz_cap) record(a.st, SA_ERR_CAPACITY, CHK_CAPACITY_CSR, (int)min(run, (long long)INT32_MAX));
+    }
+}
+
+__global__ void __launch_bounds__(kScanChunk) k_csr_scan(const RbsArgs a, const long long *chunk_off)
+{
+    pdl_wait();
+    pdl_trigger();
+    __shared__ long long wt[33];
+    const int R = a.Hq * a.nB;
+    const int r = blockIdx.x * kScanChunk + threadIdx.x;
+    long long total;
+    const long long ex = block_excl_scan_ll(r < R ? a.rowcnt[r] : 0, wt, total);
+    if (r < R) a.row_ptr[r] = (int32_t)min(chunk_off[blockIdx.x] + ex, (long long)INT32_MAX);
+}
+
+__global__ void __launch_bounds__(256) k_csr_fill(const RbsArgs a)
+{
+    pdl_wait();
+    pdl_trigger();
     if (blockIdx.x == 0 && a.tau_out)
         for (int x = threadIdx.x; x < 2 * a.Hq; x += blockDim.x) a.tau_out[x] = a.tau[x];
-    long long part = 0;
-    for (int t = threadIdx.x; t < tile; t += blockDim.x) part += a.tilecnt[t];
-    long long off;
-    block_excl_scan_ll(part, wt, off);           // off: sum over the preceding tiles
-    const int i = I * kRbsImgRows + (int)threadIdx.x;
-    const bool mine = threadIdx.x < kRbsImgRows && i < a.nB;
-    const int cnt = mine ? a.rowcnt[(size_t)h * a.nB + i] : 0;
-    long long tot;
-    const long long ex = block_excl_scan_ll(cnt, wt, tot);
-    if (mine) {
-        const long long p = off + ex;
-        a.row_ptr[(size_t)h * a.nB + i] = (int32_t)min(p, (long long)INT32_MAX);
-        s_base[threadIdx.x] = p;
-    }
-    if (tile == (int)gridDim.x - 1 && threadIdx.x == 0) {
-        const long long end = off + tot;
-        a.row_ptr[(size_t)a.Hq * a.nB] = (int32_t)min(end, (long long)INT32_MAX);
-        if (end > a.nnz_cap) record(a.st, SA_ERR_CAPACITY, CHK_CAPACITY_CSR, (int)min(end, (long long)INT32_MAX));
-    }
-    __syncthreads();
-    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= a.Hq * a.nB) return;
+    const int i = row % a.nB;
     const int words = rbs_mask_words(a.nB);
-    for (int rr = warp; rr < kRbsImgRows; rr += 8) {
-        const int ii = I * kRbsImgRows + rr;
-        if (ii >= a.nB) break;
-        const size_t row = (size_t)h * a.nB + ii;
-        const int nw = ii / 32 + 1;
-        long long base = s_base[rr];
-        for (int w0 = 0; w0 < nw; w0 += 32) {
-            const int w = w0 + lane;
-            const uint32_t bits = w < nw ? a.bits[row * words + w] : 0u;
-            const int c = __popc(bits);
-            int pre = c;
+    const int nw = i / 32 + 1;
+    long long base = a.row_ptr[row];
+    for (int w0 = 0; w0 < nw; w0 += 32) {
+        const int w = w0 + lane;
+        const uint32_t bits = w < nw ? a.bits[(size_t)row * words + w] : 0u;
+        const int c = __popc(bits);
+        int pre = c;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, pre, o);
-                if (lane >= o) pre += y;
-            }
-            const int tw = __shfl_sync(0xffffffffu, pre, 31);
-            long long pos = base + pre - c;
-            uint32_t b = bits;
-            while (b) {
-                const int bit = __ffs(b) - 1;
-                b &= b - 1;
-                if (pos < a.nnz_cap) a.cols[pos] = w * 32 + bit;
-                ++pos;
-            }
-            base += tw;
+        for (int o = 1; o < 32; o <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, pre, o);
+            if (lane >= o) pre += y;
         }
+        const int tot = __shfl_sync(0xffffffffu, pre, 31);
+        long long pos = base + pre - c;
+        uint32_t b = bits;
+        while (b) {
+            const int bit = __ffs(b) - 1;
+            b &= b - 1;
+            if (pos < a.nnz_cap) a.cols[pos] = w * 32 + bit;
+            ++pos;
+        }
+        base += tot;
     }
 }
 
@@ -508,8 +514,15 @@ cudaError_t launch_rbs(const RbsArgs &a, cudaStream_t s)
         if ((e = launch_pair_tc(a, false, s)) != cudaSuccess) return e;
     }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    const int nTB = rbs_img_tiles(a.nB);
-    if (cudaError_t e_ = launch_pdl(k_csr_fill, dim3(a.Hq * nTB), dim3(256), 0, s, a, nTB)) return e_;
+    {
+        const int R = a.Hq * a.nB;
+        const int nch = (R + kScanChunk - 1) / kScanChunk;
+        long long *chunk = reinterpret_cast<long long *>(a.rowcnt + R + 1 + ((R + 1) & 1));   // 8-byte aligned
+        if (cudaError_t e_ = launch_pdl(k_csr_sum, dim3(nch), dim3(kScanChunk), 0, s, a, chunk)) return e_;
+        if (cudaError_t e_ = launch_pdl(k_csr_chunks, dim3(1), dim3(1024), 0, s, a, chunk, nch)) return e_;
+        if (cudaError_t e_ = launch_pdl(k_csr_scan, dim3(nch), dim3(kScanChunk), 0, s, a, chunk)) return e_;
+    }
+    if (cudaError_t e_ = launch_pdl(k_csr_fill, dim3((a.Hq * a.nB + 7) / 8), dim3(256), 0, s, a)) return e_;
     return cudaGetLastError();
 }
 

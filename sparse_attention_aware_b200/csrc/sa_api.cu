@@ -354,7 +354,6 @@ sa_status sa_select_blocks(const sa_kv_cache *kv, const sa_block_select_args *ar
     a.tau = reinterpret_cast<float *>(w + offs[4]);
     a.bits = reinterpret_cast<uint32_t *>(w + offs[5]);
     a.rowcnt = reinterpret_cast<int32_t *>(w + offs[6]);
-    a.tilecnt = a.rowcnt + (size_t)Hq * nB;
     a.pair_sc = quant ? reinterpret_cast<float *>(w + offs[7]) : nullptr;
     a.qhist = quant ? reinterpret_cast<uint32_t *>(w + offs[8]) : nullptr;
     a.row_ptr = out->row_ptr;

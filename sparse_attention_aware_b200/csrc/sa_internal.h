@@ -104,8 +104,7 @@ struct RbsArgs {
     float *qnorm;    // [Hq][nB]
     float *tau;      // [2][Hq] thresholds in use
     uint32_t *bits;  // [Hq][nB][rbs_mask_words(nB)] mask bits
-    int32_t *rowcnt; // [Hq*nB] kept pairs per row
-    int32_t *tilecnt;// [Hq][rbs_img_tiles(nB)] kept pairs per 128-row tile
+    int32_t *rowcnt; // [Hq*nB]
     float *pair_sc;  // quantile mode: [Hq][nP] S_c, [Hq][nP] S_r
     uint32_t *qhist; // quantile mode scratch
     // outputs
