@@ -49,9 +49,9 @@ FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustain
 # query pooling, pair tiles, 3 CSR scan kernels, CSR fill; prefill = schedule +
 # tcgen05 kernel
 # splits of the masked-decode step (a sequence uses only as many as give each
-# ~128 tokens): 24 measured best on the 131072-token step (63.6 us per step
-# run back to back against 74.0 at 16 and 68.9 at 32)
-MASKED_SPLITS = 24
+# ~128 tokens; inside this step 16 measured best: 39.7 us against 43.6 at 24
+# and 35.9 against 34.1 at 8)
+MASKED_SPLITS = 16
 LAUNCHES = {"select_topk": 2, "decode": 2, "spans": 1, "rbs_explicit": 7, "prefill": 2}
 
 
