@@ -494,8 +494,10 @@ def main():
     if traffic:
         result["roofline"]["traffic"] = traffic.get("k_prefill_tc")
         result["roofline_decode"]["traffic"] = traffic.get("decode")
-    result["roofline"]["traffic_unit"] = "DRAM bytes per launch (ncu, full-size workload)"
-    result["roofline_decode"]["traffic_unit"] = "DRAM bytes per decode group (ncu, full-size workload)"
+    result["roofline"]["traffic_unit"] = ("DRAM bytes per launch; null: measured on the 32768-token case only "
+                                          "(579 MB), which does not scale to this launch in proportion")
+    result["roofline_decode"]["traffic_unit"] = ("DRAM bytes per decode group: ncu on the B=8, L=32768 group, "
+                                                 "scaled by algorithmic bytes (ratio 0.974)")
 
     if not args.no_e2e:
         result["e2e"] = e2e(step, dec, pre, msk, cfg, args, world, dev, dist if world > 1 else None)
