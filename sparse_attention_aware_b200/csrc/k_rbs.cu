@@ -64,7 +64,9 @@ __device__ __forceinline__ void store_split(uint8_t *img, int row, int k, float 
 }
 
 // ---------------------------------------------------------------------------
-// Block statistics (one CTA per key block and kv head) and query pooling (one
+// Block statistics (one CTA per key block and kv head; the block's rows stay
+// in registers: column sums, then squared distances from the centroid) and
+// query pooling (one
 // CTA per query block and q head), two launches over nB rounded up to whole
 // 128-row tile images, whose padding rows are zeroed.  The pooling CTA of
 // (i, h) also clears row i's mask count of head h, and the first statistics
@@ -72,11 +74,9 @@ __device__ __forceinline__ void store_split(uint8_t *img, int row, int k, float 
 // CTA was measured 10% slower.)
 // ---------------------------------------------------------------------------
 struct StatsSmem {
-    uint16_t tile[BS * 128];   // key block, bf16 rows
+    float csum[8][128];        // per-warp column sums
     float cen[128];
-    float csum[2][128];
     float wmax[8];
-    int page[BS];              // physical page of each page of the block (<= 64 pages)
 };
 struct PoolSmem {
     float part[16][128];
@@ -98,73 +98,83 @@ __device__ void block_stats_cta(const RbsArgs &a, StatsSmem &sm, int j, int g)
     }
     const int n = min(BS, a.T - j * BS);
     const int P = 1 << a.c.Plog2;
-    // pages of the block (one at P = 64): looked up once, not per row
-    const int npg = (n + P - 1) >> a.c.Plog2;
-    if (threadIdx.x < npg) {
-        int page = __ldg(a.c.pt + ((j * BS) >> a.c.Plog2) + threadIdx.x);
-        if (page < 0 || page >= a.c.num_pages) {
-            fault(a.st, CHK_PAGE, page);
-            page = -1;
-        }
-        sm.page[threadIdx.x] = page;
-    }
-    __syncthreads();
-    // stage the block's rows: 16-byte chunks, all of a thread's loads in flight at once
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int c8 = tid & 15;                 // this thread's 8 columns: 8*c8 ..
+    // rows (tid >> 4) + 16u, u = 0..3, held in registers (16-byte loads, all
+    // in flight at once); the block starts on a page edge (P divides 64)
     uint4 v[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-        const int ch = threadIdx.x + u * 256;   // 64 rows x 16 chunks = 1024
-        const int r = ch >> 4, c8 = ch & 15;
+        const int r = (tid >> 4) + 16 * u;
         v[u] = make_uint4(0, 0, 0, 0);
         if (r < n) {
-            const int page = sm.page[r >> a.c.Plog2];
-            if (page >= 0) {
-                const size_t off = ((((size_t)page * a.c.Hkv + g) << a.c.Plog2) + (r & (P - 1))) * D + c8 * 8;
+            int page = __ldg(a.c.pt + ((j * BS + r) >> a.c.Plog2));
+            if (page < 0 || page >= a.c.num_pages) {
+                fault(a.st, CHK_PAGE, page);
+            } else {
+                const size_t off = ((((size_t)page * a.c.Hkv + g) << a.c.Plog2) + ((j * BS + r) & (P - 1))) * D + c8 * 8;
                 v[u] = ldg_nc_v4(a.c.k + off);
             }
         }
     }
+    // column sums: the thread's rows, then the other row group of the warp
+    // (lane ^ 16 holds the same columns), then the eight warps via shared memory
+    float cs[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) cs[e] = 0.f;
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-        const int ch = threadIdx.x + u * 256;
-        *reinterpret_cast<uint4 *>(&sm.tile[(ch >> 4) * D + (ch & 15) * 8]) = v[u];
-    }
-    __syncthreads();
-    {   // column sums: two threads per column, rows interleaved, 4 chains each
-        const int col = threadIdx.x & (D - 1), half = threadIdx.x >> 7;
-        float s4[4] = {0.f, 0.f, 0.f, 0.f};
-        for (int r = half; r < n; r += 8)
-#pragma unroll
-            for (int q = 0; q < 4; ++q)
-                if (r + 2 * q < n) s4[q] += __uint_as_float((uint32_t)sm.tile[(r + 2 * q) * D + col] << 16);
-        sm.csum[half][col] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
-    }
-    __syncthreads();
-    if (threadIdx.x < D) {
-        const float c = (sm.csum[0][threadIdx.x] + sm.csum[1][threadIdx.x]) / (float)n;
-        sm.cen[threadIdx.x] = c;
-        store_split(img, j & 127, threadIdx.x, c);
-    }
-    __syncthreads();
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    float mx = 0.f;
-    for (int r = warp; r < n; r += 8) {
-        float e = 0.f;
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
-            const int col = lane * 4 + q;
-            const float dlt = __uint_as_float((uint32_t)sm.tile[r * D + col] << 16) - sm.cen[col];
-            e = fmaf(dlt, dlt, e);
+            cs[2 * q] += bf_lo(w[q]);
+            cs[2 * q + 1] += bf_hi(w[q]);
         }
-        e = warp_sum(e);
-        mx = fmaxf(mx, sqrtf(e));
     }
+#pragma unroll
+    for (int e = 0; e < 8; ++e) cs[e] += __shfl_xor_sync(0xffffffffu, cs[e], 16);
+    if (lane < 16) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) sm.csum[warp][8 * c8 + e] = cs[e];
+    }
+    __syncthreads();
+    if (tid < D) {
+        float t = 0.f;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) t += sm.csum[w][tid];
+        const float c = t / (float)n;
+        sm.cen[tid] = c;
+        store_split(img, j & 127, tid, c);
+    }
+    __syncthreads();
+    // max radius: squared distance of each row from the centroid, summed over
+    // the 16 lanes that hold the row, max over rows; sqrt is monotone, so the
+    // root of the largest square is the largest radius
+    float cc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) cc[e] = sm.cen[8 * c8 + e];
+    float mx = 0.f;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        float d = 0.f;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            const float x0 = bf_lo(w[q]) - cc[2 * q], x1 = bf_hi(w[q]) - cc[2 * q + 1];
+            d = fmaf(x0, x0, d);
+            d = fmaf(x1, x1, d);
+        }
+#pragma unroll
+        for (int o = 8; o > 0; o >>= 1) d += __shfl_xor_sync(0xffffffffu, d, o);
+        if ((tid >> 4) + 16 * u < n) mx = fmaxf(mx, d);
+    }
+    mx = warp_max(mx);
     if (lane == 0) sm.wmax[warp] = mx;
     __syncthreads();
-    if (threadIdx.x == 0) {
+    if (tid == 0) {
         float m = 0.f;
         for (int w = 0; w < 8; ++w) m = fmaxf(m, sm.wmax[w]);
-        a.rad[(size_t)g * rad_rows + j] = m;
+        a.rad[(size_t)g * rad_rows + j] = sqrtf(m);
     }
 }
 
