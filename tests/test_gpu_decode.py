@@ -249,3 +249,35 @@ def test_bench_decode_config(cuda_dev):
         assert_close_attn(out.float().cpu().numpy().reshape(-1, 128)[rows], ref)
         np.testing.assert_allclose(lse.cpu().numpy().reshape(-1)[rows], ref_lse, atol=2e-3, rtol=0)
     ws.raise_on_fault()
+
+
+def test_default_workspaces_are_per_stream(cuda_dev):
+    """Calls without an explicit workspace on two streams get separate default
+    workspaces, so decodes queued on both streams at once do not share
+    split-KV scratch: each equals the same decode run alone."""
+    import sparse_attention_aware_b200.api as api
+    cache, q = W.random_decode(31, 4, 16, 4, 128, [3000, 1777, 4096, 900], 16)
+    gc, qd = cache.to(cuda_dev), q.to(cuda_dev)
+    rng = np.random.default_rng(31)
+    sels = []
+    for seed in (1, 2):
+        idx = np.full((4, 16, 512), -1, dtype=np.int32)
+        cnt = np.zeros((4, 16), dtype=np.int32)
+        for b, L in enumerate([3000, 1777, 4096, 900]):
+            for h in range(16):
+                n = int(rng.integers(1, 512))
+                idx[b, h, :n] = np.sort(rng.choice(L, n, replace=False))
+                cnt[b, h] = n
+        sels.append(sa.TokenSelection(torch.from_numpy(idx).to(cuda_dev), torch.from_numpy(cnt).to(cuda_dev)))
+    want = [sa.sparse_decode_attn(gc, qd, s, 0.09, 8, ws=sa.Workspace(cuda_dev))[0] for s in sels]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(cuda_dev), torch.cuda.Stream(cuda_dev)]
+    got = [None, None]
+    for rep in range(3):
+        for i, s in enumerate(streams):
+            got[i] = sa.sparse_decode_attn(gc, qd, sels[i], 0.09, 8, stream=s)[0]
+        torch.cuda.synchronize()
+        for i in range(2):
+            assert torch.equal(got[i], want[i])
+    keys = [k for k in api._default_ws if k[0] == str(cuda_dev)]
+    assert {k[1] for k in keys} >= {int(s.cuda_stream) for s in streams}
