@@ -142,6 +142,13 @@ class TieredKV:
         self.mirror_free = [None, None]
         self.flip = 0
         self.dev_pt = torch.full(self.host_pt.shape, -1, dtype=torch.int32, device=self.device)
+        # (host page, slot) fetch lists: two pinned host buffers used alternately
+        # (a pinned allocation per step costs milliseconds) and one device
+        # buffer, rewritten on the copy stream after the previous fetch read it
+        self.pairs_host = [torch.zeros((slots, 2), dtype=torch.int32).pin_memory() for _ in range(2)]
+        self.pairs_free = [None, None]
+        self.pflip = 0
+        self.pairs_dev = torch.zeros((slots, 2), dtype=torch.int32, device=self.device)
         self.stream = copy_stream or torch.cuda.Stream(self.device)
         self.ws = api.Workspace(self.device)
         self.ready = torch.cuda.Event()
@@ -210,7 +217,17 @@ class TieredKV:
             if self.prev_mark is not None:
                 self.stream.wait_event(self.prev_mark)
             if pairs:
-                pr = torch.tensor(pairs, dtype=torch.int32).pin_memory().to(self.device, non_blocking=True)
+                n = len(pairs)
+                hb = self.pflip
+                self.pflip ^= 1
+                if self.pairs_free[hb] is not None:
+                    self.pairs_free[hb].synchronize()     # its copy two fetches ago is done
+                self.pairs_host[hb].numpy()[:n] = np.asarray(pairs, dtype=np.int32)
+                pr = self.pairs_dev[:n]
+                pr.copy_(self.pairs_host[hb][:n], non_blocking=True)
+                done_p = torch.cuda.Event()
+                done_p.record(self.stream)
+                self.pairs_free[hb] = done_p
                 if self.time_fetches:
                     ev = (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                     ev[0].record(self.stream)
