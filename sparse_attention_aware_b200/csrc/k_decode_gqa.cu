@@ -7,58 +7,51 @@
 // segments per sequence, shared by every head.  So the query heads of a GQA
 // group read the same K/V rows, and with 8 heads per kv head the work is
 // ~8 flop per byte of K/V -- at the limit of fp32 SIMT issue, so the two
-// contractions (Q K^T and P V) go to the tensor cores with the group's heads
-// as the M rows of an m16n8k16 MMA.  Partials per split are merged by the
+// contractions go to the tensor cores.  Partials per split are merged by the
 // common combine kernel ("稀疏注意力机制创新…", section "四、从外卖到AI":
 // SplitKV-and-Combine).
 //
-// One CTA = (split s, kv head g, sequence b), 4 warps.  The split owns a
+// One CTA = (split s, kv head g, sequence b), kPW warps.  The split owns a
 // contiguous range of the sequence's list entries (balanced by entry count;
 // an entry is at most one page); a sequence uses only as many of the S splits
-// as give each at least ~128 tokens.  Entries are staged in shared memory in
-// windows of up to kWin, validated, mapped to physical pages once, and
-// prefix-summed into positions; each entry's K and V rows are prefetched into
-// L2 right away (one bulk prefetch each), so the latency of the scattered page
-// reads is paid about once per CTA, not once per tile.  64-token tiles of K and V rows are gathered
-// with 16-byte cp.async into a double-buffered, XOR-swizzled tile (rows of
-// D*2 bytes; 16-byte chunk c of row r lives at chunk c ^ (r & 7), so the
-// 8-row ldmatrix reads are free of bank conflicts).  Warp w owns tokens
-// [16w, 16w + 16) of a tile: S = Q K^T (fp32 accumulate; an fp32 query is
-// split into bf16 high and low parts, two MMAs), online softmax per head in
-// the base-2 domain, P as bf16, O += P V.  The warps' states are merged
-// through shared memory at the end and written as one split partial.
+// as give each at least ~128 tokens.  The warps take the split's entries
+// round-robin and run independently until the final merge: a warp holds up
+// to 32 of its entries in registers (one per lane: validated, page-mapped)
+// and walks them as pieces of at most 16 consecutive rows of one page.  A
+// piece's 16 K rows and 16 V rows are fetched by 32 bulk copies (one row per
+// lane; rows past the entry's end repeat its last row, so every piece is
+// 16 finite rows and its probability is 0 there) into the warp's kNST-stage
+// ring, rows padded to D*2 + 16 bytes so that 8-row ldmatrix reads hit 32
+// distinct banks; each stage completes on its own mbarrier.
+//
+// The contractions take the 16 tokens of a piece as the M rows and the
+// group's heads as the N columns of m16n8k16 (no padding rows for 8 heads):
+// S^T = K Q^T (fp32 accumulate; an fp32 query is split into bf16 high and low
+// parts, two MMAs), online softmax per head (column) in the base-2 domain,
+// P^T as bf16 moved into the B-operand layout with movmatrix, then
+// O^T += V^T P^T with V^T read by transposing ldmatrix.
 #include "sa_internal.h"
+#include "tc_ptx.cuh"
 
 namespace sa {
 namespace {
 
-constexpr int kGT = 64;                  // tokens per tile
-constexpr int kGWarps = 4;               // a warp owns 16 tokens of a tile
-constexpr int kGThreads = kGWarps * 32;
-constexpr int kWin = 512;                // list entries staged per window
+constexpr int kPW = 4;                   // warps per CTA
+constexpr int kGThreads = kPW * 32;
+constexpr int kPR = 16;                  // rows per piece (the MMA's M)
+constexpr int kNST = 2;                  // ring stages per warp
 constexpr int kSplitTokens = 128;        // a split of a sequence's list covers at least ~this many tokens
+constexpr uint64_t kGqaWaitNs = 1000ull * 1000 * 1000;   // 1 s
 
 template <int D>
 struct GqaSmem {
-    static constexpr int TILE = kGT * D * 2;                   // one K or V tile, bytes
-    static constexpr int KV = 2 * 2 * TILE;                    // K and V, double buffered
-    static constexpr int MERGE = kGWarps * (16 * D + 32) * 4;  // per-warp O, m, l
-    static constexpr int BODY = KV > MERGE ? KV : MERGE;
-    static constexpr int ENT = kWin * 16 + (kWin + 1) * 4 + kGT * 2 * 4 + 16;   // went, pre, rowok, total
-    static constexpr int BYTES = BODY + ENT;
+    static constexpr int ROW = D * 2 + 16;                      // padded row, bytes
+    static constexpr int STAGE = 2 * kPR * ROW;                 // K rows, then V rows
+    static constexpr int RING = kPW * kNST * STAGE;
+    static constexpr int MERGE = kPW * (16 * D + 32) * 4;       // per-warp O, m, l (up to 16 heads)
+    static constexpr int BODY = RING > MERGE ? RING : MERGE;
+    static constexpr int BYTES = BODY + kPW * kNST * 8 + 16;    // + mbarriers, abort flag
 };
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src, bool pred)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(pred ? 16 : 0)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait()
-{
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2, uint32_t &r3)
 {
@@ -72,6 +65,13 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t 
                  : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                  : "r"(addr));
 }
+// transpose of an 8x8 b16 matrix held in the mma fragment layout
+__device__ __forceinline__ uint32_t movm_t(uint32_t x)
+{
+    uint32_t y;
+    asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(y) : "r"(x));
+    return y;
+}
 
 // D (16x8 fp32) += A (16x16 bf16, row) * B (16x8 bf16, col)
 __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1)
@@ -83,12 +83,6 @@ __device__ __forceinline__ void mma16816(float (&d)[4], const uint32_t (&a)[4], 
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-// start moving `bytes` (a multiple of 16, 16-byte aligned) into L2
-__device__ __forceinline__ void prefetch_l2(const void *p, uint32_t bytes)
-{
-    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
-}
-
 __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi)
 {
     return (uint32_t)f2bf(lo) | ((uint32_t)f2bf(hi) << 16);
@@ -96,7 +90,7 @@ __device__ __forceinline__ uint32_t pack_bf2(float lo, float hi)
 
 __device__ __forceinline__ float bf_round(float x) { return __uint_as_float((uint32_t)f2bf(x) << 16); }
 
-// Query fragment words for row m (zero for padding rows), element pair
+// Query words for head row `row_off` (zero for padding heads), element pair
 // (col, col + 1): bf16 high part, and for an fp32 query also the bf16 low part
 // (x - bf16(x)), so that hi + lo carries the query to ~16 bits.
 template <bool QF32>
@@ -115,21 +109,20 @@ __device__ __forceinline__ void q_pair(const void *q, size_t row_off, bool valid
     }
 }
 
-template <int D, bool QF32>
+// NH = 8-head column blocks (1: up to 8 heads per kv head, 2: up to 16)
+template <int D, int NH, bool QF32>
 __global__ void __launch_bounds__(kGThreads) k_decode_gqa_blocks(const DecodeArgs a)
 {
     pdl_wait();
     pdl_trigger();
     using SM = GqaSmem<D>;
-    constexpr int KK = D / 16;   // k-steps of Q K^T
-    constexpr int NB = D / 8;    // n-blocks of the output
-    constexpr int CH = D / 8;    // 16-byte chunks per row
+    constexpr int KK = D / 16;   // k-steps of S^T = K Q^T
+    constexpr int MT = D / 16;   // m-tiles of O^T
+    constexpr int NQ = QF32 ? 2 : 1;
     extern __shared__ __align__(128) uint8_t sm[];
     const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(sm);
-    int4 *went = reinterpret_cast<int4 *>(sm + SM::BODY);             // [kWin] {lo, len, page, -}
-    int *pre = reinterpret_cast<int *>(sm + SM::BODY + kWin * 16);    // [kWin + 1] first position
-    int *rowok = pre + kWin + 1;                                       // [2][kGT]
-    int *s_tot = rowok + 2 * kGT;
+    uint64_t *bars = reinterpret_cast<uint64_t *>(sm + SM::BODY);   // [kPW][kNST]
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + kPW * kNST);
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int gq = lane >> 2, tq = lane & 3;   // mma group id / thread in group
@@ -167,240 +160,244 @@ __global__ void __launch_bounds__(kGThreads) k_decode_gqa_blocks(const DecodeArg
     const int32_t *ptb = a.c.pt + (size_t)b * a.c.max_pages;
     const int P = 1 << a.c.Plog2;
 
-    // query fragments: rows m = gq and gq + 8 are heads g*HPG + m when m < HPG
-    uint32_t qa[KK][4], ql[QF32 ? KK : 1][4];
-    {
-        const size_t r0 = ((size_t)b * a.Hq + g * HPG + gq) * D;
-        const size_t r1 = r0 + (size_t)8 * D;
-        const bool v0 = gq < HPG, v1 = gq + 8 < HPG;
+    if (tid == 0) {
+        for (int i = 0; i < kPW * kNST; ++i) tc::mbar_init(bars + i, 1);
+        *abort_flag = 0;
+        tc::fence_mbar_init();
+    }
+
+    // query B fragments: column n of block nh is head nh*8 + gq (zero past HPG);
+    // k pairs (2tq, 2tq+1) and (2tq+8, 2tq+9) of k-step kk
+    uint32_t qb[NQ][NH][KK][2];
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh) {
+        const int h = nh * 8 + gq;
+        const size_t r0 = ((size_t)b * a.Hq + g * HPG + h) * D;
+        const bool v = h < HPG;
 #pragma unroll
         for (int kk = 0; kk < KK; ++kk) {
-            const int c = kk * 16 + 2 * tq;
-            uint32_t lo[4];
-            q_pair<QF32>(a.q, r0, v0, c, qa[kk][0], lo[0]);
-            q_pair<QF32>(a.q, r1, v1, c, qa[kk][1], lo[1]);
-            q_pair<QF32>(a.q, r0, v0, c + 8, qa[kk][2], lo[2]);
-            q_pair<QF32>(a.q, r1, v1, c + 8, qa[kk][3], lo[3]);
+            uint32_t lo0, lo1;
+            q_pair<QF32>(a.q, r0, v, kk * 16 + 2 * tq, qb[0][nh][kk][0], lo0);
+            q_pair<QF32>(a.q, r0, v, kk * 16 + 2 * tq + 8, qb[0][nh][kk][1], lo1);
             if (QF32) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) ql[QF32 ? kk : 0][i] = lo[i];
+                qb[NQ - 1][nh][kk][0] = lo0;
+                qb[NQ - 1][nh][kk][1] = lo1;
             }
         }
     }
+    __syncthreads();   // mbarriers initialised
 
-    float o[NB][4];
+    // O^T fragments: o[mt][nh][i] = O[head nh*8 + 2tq + (i & 1)][d = mt*16 + gq + 8*(i >> 1)]
+    float o[MT][NH][4];
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) o[nb][0] = o[nb][1] = o[nb][2] = o[nb][3] = 0.f;
-    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;   // rows gq, gq + 8 (l: this thread's part)
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nh = 0; nh < NH; ++nh) o[mt][nh][0] = o[mt][nh][1] = o[mt][nh][2] = o[mt][nh][3] = 0.f;
+    float mh[NH][2], lh[NH][2];   // heads nh*8 + 2tq + j (l: this thread's tokens only)
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh) mh[nh][0] = mh[nh][1] = -INFINITY, lh[nh][0] = lh[nh][1] = 0.f;
 
-    for (int wb = e0; wb < e1; wb += kWin) {
-        const int nE = min(kWin, e1 - wb);
-        __syncthreads();   // previous window's tiles are done with went / pre
-        // stage, validate and map the window's entries; lengths into pre[]
-        for (int i = tid; i < nE; i += kGThreads) {
-            const int4 en = ent[wb + i];
-            const int x = en.x, lo = en.y, hi = en.z;
-            bool ok = lo >= 0 && lo < hi && hi <= P && x >= 0 && x < a.c.max_pages;
-            if (!ok) fault(st, CHK_BLOCK_ENTRY, wb + i);
+    uint64_t *wbar = bars + warp * kNST;
+    const uint32_t wring = sbase + warp * kNST * SM::STAGE;
+    uint8_t *wring_g = sm + warp * kNST * SM::STAGE;
+    const uint64_t deadline = tc::globaltimer() + kGqaWaitNs;
+    int gpc = 0;          // pieces this warp has consumed (stage = gpc % kNST, parity = (gpc / kNST) & 1)
+    bool alive = true;
+
+    // this warp's entries: e0 + warp + kPW * j
+    for (int wb = e0 + warp; wb < e1 && alive; wb += 32 * kPW) {
+        // one entry per lane: validate and map (len 0 = skipped)
+        const int e = wb + kPW * lane;
+        int pg = 0, lo = 0, len = 0;
+        if (e < e1) {
+            const int4 en = ent[e];
+            const int x = en.x, l0 = en.y, hi = en.z;
+            bool ok = l0 >= 0 && l0 < hi && hi <= P && x >= 0 && x < a.c.max_pages;
+            if (!ok) fault(st, CHK_BLOCK_ENTRY, e);
             if (ok && (x << a.c.Plog2) + hi > L) {
                 fault(st, CHK_INDEX, (x << a.c.Plog2) + hi - 1);
                 ok = false;
             }
-            int page = 0;
             if (ok) {
-                page = __ldg(ptb + x);
-                if (page < 0 || page >= a.c.num_pages) {
-                    fault(st, CHK_PAGE, page);
+                pg = __ldg(ptb + x);
+                if (pg < 0 || pg >= a.c.num_pages) {
+                    fault(st, CHK_PAGE, pg);
                     ok = false;
                 }
             }
-            went[i] = make_int4(lo, ok ? hi - lo : 0, page, 0);
             if (ok) {
-                // the tiles read this entry's rows one after another: start all
-                // of them towards L2 now, so that only the first tile waits on DRAM
-                const size_t off = ((((size_t)page * a.c.Hkv + g) << a.c.Plog2) + lo) * D;
-                prefetch_l2(a.c.k + off, (uint32_t)(hi - lo) * D * 2);
-                prefetch_l2(a.c.v + off, (uint32_t)(hi - lo) * D * 2);
+                lo = l0;
+                len = hi - l0;
             }
         }
-        __syncthreads();
-        if (warp == 0) {
-            // exclusive prefix of the lengths (serial over 32-entry runs per lane)
-            const int per = (nE + 31) / 32;
-            const int i0 = min(lane * per, nE), i1 = min(i0 + per, nE);
-            int run = 0;
-            for (int i = i0; i < i1; ++i) run += went[i].y;
-            int incl = run;
+        // pieces per entry, inclusive prefix over the lanes
+        const int npc = (len + kPR - 1) / kPR;
+        int incl = npc;
 #pragma unroll
-            for (int off = 1; off < 32; off <<= 1) {
-                const int y = __shfl_up_sync(0xffffffffu, incl, off);
-                if (lane >= off) incl += y;
-            }
-            int base = incl - run;
-            for (int i = i0; i < i1; ++i) {
-                pre[i] = base;
-                base += went[i].y;
-            }
-            if (lane == 31) *s_tot = incl;
+        for (int off = 1; off < 32; off <<= 1) {
+            const int y = __shfl_up_sync(0xffffffffu, incl, off);
+            if (lane >= off) incl += y;
         }
-        __syncthreads();
-        const int nw = *s_tot;
-        const int ntile = (nw + kGT - 1) / kGT;
+        const int np = __shfl_sync(0xffffffffu, incl, 31);
 
-        // gather: thread -> (row r, half of the row's chunks), K and V
-        auto issue = [&](int tile, int buf) {
-            const int r = tid >> 1;
-            const int p = tile * kGT + r;
-            const bool ok = p < nw;
-            size_t src = 0;
-            if (ok) {
-                int lo = 0, hi = nE - 1;   // last entry with pre[e] <= p
-                while (lo < hi) {
-                    const int mid = (lo + hi + 1) >> 1;
-                    if (pre[mid] <= p) lo = mid; else hi = mid - 1;
-                }
-                const int4 en = went[lo];
-                const int tok = en.x + (p - pre[lo]);
-                src = ((((size_t)en.z * a.c.Hkv + g) << a.c.Plog2) + tok) * D;
-            }
-            if ((tid & 1) == 0) rowok[buf * kGT + r] = ok ? 1 : 0;
-            const uint32_t kd = sbase + buf * SM::TILE + r * D * 2;
-            const uint32_t vd = sbase + 2 * SM::TILE + buf * SM::TILE + r * D * 2;
-#pragma unroll
-            for (int j = 0; j < CH / 2; ++j) {
-                const int c = (tid & 1) * (CH / 2) + j;
-                const uint32_t sw = (uint32_t)((c ^ (r & 7)) * 16);
-                cp_async16(kd + sw, a.c.k + src + c * 8, ok);
-                cp_async16(vd + sw, a.c.v + src + c * 8, ok);
-            }
+        // piece n: lane of its entry, then its first row and row count
+        auto locate = [&](int n, size_t &row0, int &cnt) {
+            const unsigned m = __ballot_sync(0xffffffffu, incl > n);
+            const int src = __ffs(m) - 1;
+            const int e_pg = __shfl_sync(0xffffffffu, pg, src);
+            const int e_lo = __shfl_sync(0xffffffffu, lo, src);
+            const int e_len = __shfl_sync(0xffffffffu, len, src);
+            const int e_ex = __shfl_sync(0xffffffffu, incl - npc, src);
+            const int j = n - e_ex;
+            cnt = min(kPR, e_len - j * kPR);
+            row0 = (((size_t)e_pg * a.c.Hkv + g) << a.c.Plog2) + e_lo + j * kPR;
+        };
+        auto issue = [&](int n, int stage) {
+            size_t row0;
+            int cnt;
+            locate(n, row0, cnt);
+            if (lane == 0) tc::mbar_arrive_expect_tx(wbar + stage, (uint32_t)(2 * kPR * D * 2));
+            __syncwarp();
+            const int r = lane & (kPR - 1);
+            const size_t row = row0 + min(r, cnt - 1);
+            const uint16_t *src = (lane < kPR ? a.c.k : a.c.v) + row * D;
+            tc::bulk_load(wring_g + stage * SM::STAGE + (lane >> 4) * kPR * SM::ROW + r * SM::ROW, src,
+                          (uint32_t)(D * 2), wbar + stage);
         };
 
-        if (ntile > 0) issue(0, 0);
-        cp_async_commit();
-        for (int t = 0; t < ntile; ++t) {
-            const int buf = t & 1;
-            if (t + 1 < ntile) issue(t + 1, buf ^ 1);
-            cp_async_commit();
-            cp_async_wait<1>();
-            __syncthreads();
+        const int pre = min(np, kNST);
+        for (int n = 0; n < pre; ++n) issue(n, (gpc + n) % kNST);
+        int n = 0;
+        for (; n < np; ++n, ++gpc) {
+            const int stage = gpc % kNST;
+            const bool ok = __all_sync(0xffffffffu, tc::mbar_wait(wbar + stage, (uint32_t)(gpc / kNST) & 1u,
+                                                                  deadline, abort_flag));
+            if (!ok) {
+                *abort_flag = 1;
+                if (lane == 0) fault(st, CHK_WAIT, n);
+                alive = false;
+                break;
+            }
+            size_t row0_unused;
+            int cnt;
+            locate(n, row0_unused, cnt);
+            const uint32_t kt = wring + stage * SM::STAGE, vt = kt + kPR * SM::ROW;
 
-            // ---- S = Q K^T for this warp's 16 tokens (two n-blocks of 8)
-            float sc[2][4];
+            // ---- S^T = K Q^T: 16 tokens x (NH*8) heads
+            float sc[NH][4];
 #pragma unroll
-            for (int i = 0; i < 4; ++i) sc[0][i] = sc[1][i] = 0.f;
-            const uint32_t kt = sbase + buf * SM::TILE;
+            for (int nh = 0; nh < NH; ++nh) sc[nh][0] = sc[nh][1] = sc[nh][2] = sc[nh][3] = 0.f;
             {
-                const int mi = lane >> 3, ri = lane & 7;
-                const int tok = warp * 16 + ri + (mi >> 1) * 8;
-                const uint32_t rowa = kt + tok * D * 2;
+                const int mi = lane >> 3;
+                const uint32_t rowa = kt + ((mi & 1) * 8 + (lane & 7)) * SM::ROW + (mi >> 1) * 16;
 #pragma unroll
                 for (int kk = 0; kk < KK; ++kk) {
-                    const int c = kk * 2 + (mi & 1);
-                    uint32_t b00, b01, b10, b11;
-                    ldsm_x4(rowa + ((c ^ (tok & 7)) * 16), b00, b01, b10, b11);
-                    mma16816(sc[0], qa[kk], b00, b01);
-                    mma16816(sc[1], qa[kk], b10, b11);
-                    if (QF32) {
-                        mma16816(sc[0], ql[QF32 ? kk : 0], b00, b01);
-                        mma16816(sc[1], ql[QF32 ? kk : 0], b10, b11);
-                    }
+                    uint32_t ka[4];
+                    ldsm_x4(rowa + kk * 32, ka[0], ka[1], ka[2], ka[3]);
+#pragma unroll
+                    for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+                        for (int qi = 0; qi < NQ; ++qi) mma16816(sc[nh], ka, qb[qi][nh][kk][0], qb[qi][nh][kk][1]);
                 }
             }
-            // scale into the base-2 domain, mask rows that are not selected
+            // ---- online softmax per head column; rows gq (elements 0, 1) and gq + 8 (2, 3)
+            const bool ok0 = gq < cnt, ok1 = gq + 8 < cnt;
+            uint32_t pb[NH][2];
 #pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
-                const int tk = warp * 16 + nb * 8 + 2 * tq;
-                const bool ok0 = rowok[buf * kGT + tk] != 0, ok1 = rowok[buf * kGT + tk + 1] != 0;
-                sc[nb][0] = ok0 ? sc[nb][0] * a.qscale : -INFINITY;
-                sc[nb][1] = ok1 ? sc[nb][1] * a.qscale : -INFINITY;
-                sc[nb][2] = ok0 ? sc[nb][2] * a.qscale : -INFINITY;
-                sc[nb][3] = ok1 ? sc[nb][3] * a.qscale : -INFINITY;
-            }
-            // ---- online softmax, rows gq (elements 0, 1) and gq + 8 (2, 3)
-            float x0 = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
-            float x1 = fmaxf(fmaxf(sc[0][2], sc[0][3]), fmaxf(sc[1][2], sc[1][3]));
-            x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 1));
-            x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, 2));
-            x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 1));
-            x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, 2));
-            const float n0 = fmaxf(m0, x0), n1 = fmaxf(m1, x1);
-            const float b0 = n0 == -INFINITY ? 0.f : n0, b1 = n1 == -INFINITY ? 0.f : n1;
-            const float al0 = ex2(m0 - b0), al1 = ex2(m1 - b1);   // 0 while a row is still empty
-            m0 = n0;
-            m1 = n1;
-            float p[2][4];
+            for (int nh = 0; nh < NH; ++nh) {
+                const float s0 = ok0 ? sc[nh][0] * a.qscale : -INFINITY;
+                const float s1 = ok0 ? sc[nh][1] * a.qscale : -INFINITY;
+                const float s2 = ok1 ? sc[nh][2] * a.qscale : -INFINITY;
+                const float s3 = ok1 ? sc[nh][3] * a.qscale : -INFINITY;
+                float x0 = fmaxf(s0, s2), x1 = fmaxf(s1, s3);
 #pragma unroll
-            for (int nb = 0; nb < 2; ++nb) {
-                p[nb][0] = ex2(sc[nb][0] - b0);
-                p[nb][1] = ex2(sc[nb][1] - b0);
-                p[nb][2] = ex2(sc[nb][2] - b1);
-                p[nb][3] = ex2(sc[nb][3] - b1);
-            }
-            l0 = l0 * al0 + (p[0][0] + p[0][1]) + (p[1][0] + p[1][1]);
-            l1 = l1 * al1 + (p[0][2] + p[0][3]) + (p[1][2] + p[1][3]);
+                for (int off = 4; off < 32; off <<= 1) {
+                    x0 = fmaxf(x0, __shfl_xor_sync(0xffffffffu, x0, off));
+                    x1 = fmaxf(x1, __shfl_xor_sync(0xffffffffu, x1, off));
+                }
+                const float n0 = fmaxf(mh[nh][0], x0), n1 = fmaxf(mh[nh][1], x1);
+                const float b0 = n0 == -INFINITY ? 0.f : n0, b1 = n1 == -INFINITY ? 0.f : n1;
+                const float al0 = ex2(mh[nh][0] - b0), al1 = ex2(mh[nh][1] - b1);   // 0 while a head is empty
+                mh[nh][0] = n0;
+                mh[nh][1] = n1;
+                const float p0 = ex2(s0 - b0), p1 = ex2(s1 - b1), p2 = ex2(s2 - b0), p3 = ex2(s3 - b1);
+                lh[nh][0] = lh[nh][0] * al0 + (p0 + p2);
+                lh[nh][1] = lh[nh][1] * al1 + (p1 + p3);
 #pragma unroll
-            for (int nb = 0; nb < NB; ++nb) {
-                o[nb][0] *= al0;
-                o[nb][1] *= al0;
-                o[nb][2] *= al1;
-                o[nb][3] *= al1;
+                for (int mt = 0; mt < MT; ++mt) {
+                    o[mt][nh][0] *= al0;
+                    o[mt][nh][1] *= al1;
+                    o[mt][nh][2] *= al0;
+                    o[mt][nh][3] *= al1;
+                }
+                // P^T rows 0-7 / 8-15 (tokens) x 8 heads -> B fragments (k = tokens)
+                pb[nh][0] = movm_t(pack_bf2(p0, p1));
+                pb[nh][1] = movm_t(pack_bf2(p2, p3));
             }
-            // ---- O += P V: P (16 heads x 16 tokens) is the A operand
-            const uint32_t pa[4] = {pack_bf2(p[0][0], p[0][1]), pack_bf2(p[0][2], p[0][3]),
-                                    pack_bf2(p[1][0], p[1][1]), pack_bf2(p[1][2], p[1][3])};
-            const uint32_t vt = sbase + 2 * SM::TILE + buf * SM::TILE;
+            // ---- O^T += V^T P^T
             {
-                const int mi = lane >> 3, ri = lane & 7;
-                const int tok = warp * 16 + ri + (mi & 1) * 8;
-                const uint32_t rowa = vt + tok * D * 2;
+                const int mi = lane >> 3;
+                const uint32_t rowa = vt + ((mi >> 1) * 8 + (lane & 7)) * SM::ROW + (mi & 1) * 16;
 #pragma unroll
-                for (int dn = 0; dn < D / 16; ++dn) {
-                    const int c = dn * 2 + (mi >> 1);
-                    uint32_t r0, r1, r2, r3;
-                    ldsm_x4_t(rowa + ((c ^ (tok & 7)) * 16), r0, r1, r2, r3);
-                    mma16816(o[2 * dn], pa, r0, r1);
-                    mma16816(o[2 * dn + 1], pa, r2, r3);
+                for (int mt = 0; mt < MT; ++mt) {
+                    uint32_t va[4];
+                    ldsm_x4_t(rowa + mt * 32, va[0], va[1], va[2], va[3]);
+#pragma unroll
+                    for (int nh = 0; nh < NH; ++nh) mma16816(o[mt][nh], va, pb[nh][0], pb[nh][1]);
                 }
             }
-            __syncthreads();   // this buffer is refilled by the issue two tiles on
+            __syncwarp();   // every lane is done with this stage before it is refilled
+            if (n + kNST < np) issue(n + kNST, stage);
         }
-        cp_async_wait<0>();
+        if (!alive) {
+            // copies still in flight land before the CTA's shared memory is released
+            const uint64_t dl = tc::globaltimer() + kGqaWaitNs;
+            volatile int zero = 0;
+            for (int m = n; m < min(np, n + kNST); ++m, ++gpc)
+                tc::mbar_wait(wbar + gpc % kNST, (uint32_t)(gpc / kNST) & 1u, dl, &zero);
+        }
     }
 
-    // ---- merge the 4 warps' states through shared memory
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
-    l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 1);
-    l1 += __shfl_xor_sync(0xffffffffu, l1, 2);
+    // ---- merge the warps' states through shared memory
+#pragma unroll
+    for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+            for (int off = 4; off < 32; off <<= 1) lh[nh][j] += __shfl_xor_sync(0xffffffffu, lh[nh][j], off);
     __syncthreads();
     float *mo = reinterpret_cast<float *>(sm);                 // [warp][16][D]
-    float *mm = mo + kGWarps * 16 * D;                          // [warp][16]
-    float *ml = mm + kGWarps * 16;                              // [warp][16]
+    float *mm = mo + kPW * 16 * D;                              // [warp][16]
+    float *ml = mm + kPW * 16;                                  // [warp][16]
 #pragma unroll
-    for (int nb = 0; nb < NB; ++nb) {
-        const int c = nb * 8 + 2 * tq;
-        mo[(warp * 16 + gq) * D + c] = o[nb][0];
-        mo[(warp * 16 + gq) * D + c + 1] = o[nb][1];
-        mo[(warp * 16 + gq + 8) * D + c] = o[nb][2];
-        mo[(warp * 16 + gq + 8) * D + c + 1] = o[nb][3];
-    }
-    if (tq == 0) {
-        mm[warp * 16 + gq] = m0;
-        mm[warp * 16 + gq + 8] = m1;
-        ml[warp * 16 + gq] = l0;
-        ml[warp * 16 + gq + 8] = l1;
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const int h = nh * 8 + 2 * tq + (i & 1), d = mt * 16 + gq + 8 * (i >> 1);
+                mo[(warp * 16 + h) * D + d] = o[mt][nh][i];
+            }
+    if (gq == 0) {
+#pragma unroll
+        for (int nh = 0; nh < NH; ++nh)
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+                mm[warp * 16 + nh * 8 + 2 * tq + j] = mh[nh][j];
+                ml[warp * 16 + nh * 8 + 2 * tq + j] = lh[nh][j];
+            }
     }
     __syncthreads();
-    const int nrow = min(HPG, 16);
+    const int nrow = min(HPG, NH * 8);
     for (int i = tid; i < nrow * D; i += kGThreads) {
         const int j = i / D, c = i % D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kGWarps; ++w) M = fmaxf(M, mm[w * 16 + j]);
+        for (int w = 0; w < kPW; ++w) M = fmaxf(M, mm[w * 16 + j]);
         float O = 0.f, Ls = 0.f;
         if (M != -INFINITY) {
 #pragma unroll
-            for (int w = 0; w < kGWarps; ++w) {
+            for (int w = 0; w < kPW; ++w) {
                 const float mw = mm[w * 16 + j];
                 if (mw == -INFINITY) continue;
                 const float wgt = ex2(mw - M);
@@ -417,16 +414,23 @@ __global__ void __launch_bounds__(kGThreads) k_decode_gqa_blocks(const DecodeArg
     }
 }
 
-template <int D, bool QF32>
+template <int D, int NH, bool QF32>
 cudaError_t launch_gqa(const DecodeArgs &a, cudaStream_t s)
 {
     constexpr int smem = GqaSmem<D>::BYTES;
-    cudaError_t e = cudaFuncSetAttribute(k_decode_gqa_blocks<D, QF32>,
+    cudaError_t e = cudaFuncSetAttribute(k_decode_gqa_blocks<D, NH, QF32>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     dim3 grid(a.S, a.c.Hkv, a.c.B);
-    if (cudaError_t e_ = launch_pdl(k_decode_gqa_blocks<D, QF32>, dim3(grid), dim3(kGThreads), smem, s, a)) return e_;
+    if (cudaError_t e_ = launch_pdl(k_decode_gqa_blocks<D, NH, QF32>, dim3(grid), dim3(kGThreads), smem, s, a))
+        return e_;
     return cudaGetLastError();
+}
+
+template <int D, bool QF32>
+cudaError_t launch_gqa_nh(const DecodeArgs &a, cudaStream_t s)
+{
+    return a.Hq / a.c.Hkv <= 8 ? launch_gqa<D, 1, QF32>(a, s) : launch_gqa<D, 2, QF32>(a, s);
 }
 
 }  // namespace
@@ -435,8 +439,8 @@ bool decode_gqa_supported(const DecodeArgs &a) { return a.blocks && a.Hq / a.c.H
 
 cudaError_t launch_decode_gqa_split(const DecodeArgs &a, cudaStream_t s)
 {
-    if (a.c.D == 64) return a.q_f32 ? launch_gqa<64, true>(a, s) : launch_gqa<64, false>(a, s);
-    return a.q_f32 ? launch_gqa<128, true>(a, s) : launch_gqa<128, false>(a, s);
+    if (a.c.D == 64) return a.q_f32 ? launch_gqa_nh<64, true>(a, s) : launch_gqa_nh<64, false>(a, s);
+    return a.q_f32 ? launch_gqa_nh<128, true>(a, s) : launch_gqa_nh<128, false>(a, s);
 }
 
 }  // namespace sa
