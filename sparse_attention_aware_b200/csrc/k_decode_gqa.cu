@@ -165,6 +165,10 @@ __global__ void __launch_bounds__(kGThreads) k_decode_gqa_blocks(const DecodeArg
         *abort_flag = 0;
         tc::fence_mbar_init();
     }
+    // this lane's entry of the warp's first window, loaded before the query so
+    // that the two loads overlap
+    int4 en_first = make_int4(0, 0, 0, 0);
+    if (e0 + warp + kPW * lane < e1) en_first = ent[e0 + warp + kPW * lane];
 
     // query B fragments: column n of block nh is head nh*8 + gq (zero past HPG);
     // k pairs (2tq, 2tq+1) and (2tq+8, 2tq+9) of k-step kk
@@ -210,7 +214,7 @@ __global__ void __launch_bounds__(kGThreads) k_decode_gqa_blocks(const DecodeArg
         const int e = wb + kPW * lane;
         int pg = 0, lo = 0, len = 0;
         if (e < e1) {
-            const int4 en = ent[e];
+            const int4 en = wb == e0 + warp ? en_first : ent[e];
             const int x = en.x, l0 = en.y, hi = en.z;
             bool ok = l0 >= 0 && l0 < hi && hi <= P && x >= 0 && x < a.c.max_pages;
             if (!ok) fault(st, CHK_BLOCK_ENTRY, e);
