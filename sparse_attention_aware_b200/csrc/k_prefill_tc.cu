@@ -497,6 +497,7 @@ constexpr int kSchedRows = 64;
 constexpr int kSchedWords = 64;                 // bitmap words per row per chunk
 constexpr int kSchedBits = 32 * kSchedWords;    // key blocks per chunk
 constexpr int kSchedPairs = kSchedRows * (kSchedRows - 1) / 2;
+constexpr int kSchedSwaps = (kSchedRows / 2) * (kSchedRows / 2 - 1) / 2;   // pairs of pairs
 
 __device__ __forceinline__ int pair_index(int ka, int kb, int nc)
 {
@@ -513,6 +514,7 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
     __shared__ int pr_a[kSchedRows / 2], pr_b[kSchedRows / 2];
     __shared__ int s_best[kSchedRows], s_taken;
     __shared__ unsigned long long s_used;
+    __shared__ uint8_t sw_x[kSchedSwaps], sw_y[kSchedSwaps];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nQB = (a.T + 63) >> 6;
     const int G = a.Hq / a.c.Hkv;
@@ -529,13 +531,32 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
         __syncthreads();
         for (int w = tid; w < nc * kSchedWords; w += 256) bits[w / kSchedWords][w % kSchedWords] = 0u;
         __syncthreads();
-        for (int k = warp; k < nc; k += 8) {
-            const int i = i0 + k / G;
+        // the warp's rows k = warp + 8 j: lane j resolves row j's CSR extent,
+        // so the eight row-pointer loads are in flight together
+        int rb = 0, rn = 0;
+        if (lane < 8 && warp + 8 * lane < nc) {
+            const int k = warp + 8 * lane, i = i0 + k / G;
             const int32_t *c;
-            const int n = csr_row(a, (g * G + k % G) * nQB + i, i, c);
-            for (int e = lane; e < n; e += 32) {
-                const int rel = __ldg(c + e) - kb0;   // out-of-range entries are the kernel's to record
-                if (rel >= 0 && rel < kSchedBits && rel + kb0 <= i) atomicOr(&bits[k][rel >> 5], 1u << (rel & 31));
+            rn = csr_row(a, (g * G + k % G) * nQB + i, i, c);
+            rb = (int)(c - a.cols);
+        }
+        for (int j = 0; j < 8 && warp + 8 * j < nc; ++j) {
+            const int k = warp + 8 * j, i = i0 + k / G;
+            const int n = __shfl_sync(0xffffffffu, rn, j);
+            const int32_t *c = a.cols + __shfl_sync(0xffffffffu, rb, j);
+            for (int e0 = 0; e0 < n; e0 += 128) {
+                int v[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int e = e0 + 32 * u + lane;
+                    v[u] = e < n ? __ldg(c + e) : 0;
+                }
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int rel = v[u] - kb0;   // out-of-range entries are the kernel's to record
+                    if (e0 + 32 * u + lane < n && rel >= 0 && rel < kSchedBits && rel + kb0 <= i)
+                        atomicOr(&bits[k][rel >> 5], 1u << (rel & 31));
+                }
             }
         }
         __syncthreads();
@@ -584,20 +605,39 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
             }
         }
         __syncthreads();
-        if (tid == 0) {
-            unsigned long long nu = u;
-            int t = s_taken;
-            for (int x = 0; x < nc; ++x) {
-                const int y = s_best[x];
-                if (y > x && !(u >> x & 1ull) && s_best[y] == x) {
-                    pr_a[t] = x;
-                    pr_b[t] = y;
-                    ++t;
-                    nu |= (1ull << x) | (1ull << y);
-                }
+        if (warp == 0) {
+            // the mutually-best pairs (x < y) in increasing x, two rows per lane
+            bool f[2];
+            int yy[2];
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                const int x = lane + 32 * hh;
+                const int y = x < nc ? s_best[x] : -1;
+                f[hh] = x < nc && y > x && !(u >> x & 1ull) && s_best[y] == x;
+                yy[hh] = y;
             }
-            s_used = nu;
-            s_taken = t;
+            const unsigned b0 = __ballot_sync(0xffffffffu, f[0]), b1 = __ballot_sync(0xffffffffu, f[1]);
+            const unsigned lt = (1u << lane) - 1u;
+            const int t = s_taken;
+            unsigned long long mine = 0ull;
+            if (f[0]) {
+                const int p = t + __popc(b0 & lt);
+                pr_a[p] = lane;
+                pr_b[p] = yy[0];
+                mine |= (1ull << lane) | (1ull << yy[0]);
+            }
+            if (f[1]) {
+                const int p = t + __popc(b0) + __popc(b1 & lt);
+                pr_a[p] = lane + 32;
+                pr_b[p] = yy[1];
+                mine |= (1ull << (lane + 32)) | (1ull << yy[1]);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) mine |= __shfl_xor_sync(0xffffffffu, mine, o);
+            if (lane == 0) {
+                s_used = u | mine;
+                s_taken = t + __popc(b0) + __popc(b1);
+            }
         }
         __syncthreads();
     }
@@ -624,15 +664,21 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
     // none does
     const int npr = nc / 2, nsw = npr * (npr - 1) / 2;
     auto cst = [&](int x, int y) { return cost[x < y ? pair_index(x, y, nc) : pair_index(y, x, nc)]; };
+    // exchange q <-> pairs (x, y), x < y, in the order (0,1), (0,2), ..., (1,2), ...
+    for (int q = tid; q < nsw; q += 256) {
+        int x = 0, rem = q;
+        while (rem >= npr - 1 - x) {
+            rem -= npr - 1 - x;
+            ++x;
+        }
+        sw_x[q] = (uint8_t)x;
+        sw_y[q] = (uint8_t)(x + 1 + rem);
+    }
+    __syncthreads();
     for (int it = 0; it < 4 * kSchedRows; ++it) {
         int bg = 0, bq = INT_MAX;   // best gain (> 0), its exchange index and kind (bit 0)
         for (int q = tid; q < nsw; q += 256) {
-            int x = 0, rem = q;
-            while (rem >= npr - 1 - x) {
-                rem -= npr - 1 - x;
-                ++x;
-            }
-            const int y = x + 1 + rem;
+            const int x = sw_x[q], y = sw_y[q];
             const int ax = pr_a[x], bx = pr_b[x], ay = pr_a[y], by = pr_b[y];
             const int cur = cst(ax, bx) + cst(ay, by);
             const int o1 = cst(ax, ay) + cst(bx, by), o2 = cst(ax, by) + cst(bx, ay);
@@ -666,12 +712,7 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
         __syncthreads();                 // every thread has read red_*
         if (bg <= 0) break;              // uniform: every thread reduced the same values
         if (tid == 0) {
-            int x = 0, rem = bq >> 1;
-            while (rem >= npr - 1 - x) {
-                rem -= npr - 1 - x;
-                ++x;
-            }
-            const int y = x + 1 + rem;
+            const int x = sw_x[bq >> 1], y = sw_y[bq >> 1];
             const int bx = pr_b[x];
             if ((bq & 1) == 0) {         // (ax, ay), (bx, by)
                 pr_b[x] = pr_a[y];
