@@ -554,7 +554,7 @@ def tiered_measure(msk, cfg, dev, steps=64, slot_frac=0.125):
             mach.observe(tokens(i, b))
             lists.append(mach.next_spans(lens[b]))
         spans, cnt, rnd = packer.pack(lists)
-        tier.prepare([T.span_pages(l, n, P) for l, n in zip(lists, lens)], seq_lens=lens)
+        tier.prepare_spans(lists, lens)
         c = tier.cache
         sel = sa.select_blocks_spans(c, spans, cnt, rnd, ws=ws)
         sa.sparse_decode_attn(c, msk.q_steps[i % msk.q_steps.shape[0]], sel, 1 / math.sqrt(m["d"]), 8,

@@ -350,6 +350,37 @@ SA_API sa_status sa_fetch_pages(const void *host_k, const void *host_v, void *de
                                 size_t page_bytes, void *ws, size_t ws_bytes, sa_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* 5b. sa_tier_plan -- host-side slot planning for a tiered KV cache        */
+/* ------------------------------------------------------------------------ */
+/*
+ * [DA-1], [DA-2] as for sa_fetch_pages: before a step, the host pages it reads
+ * are mapped onto the fixed pool of device page slots.  Host code only (no GPU
+ * work, no stream); the caller's state arrays are updated in place:
+ *   slot_of   int32 [host_pages]  slot holding each host page, -1 if none
+ *   page_in   int32 [slots]       host page in each slot, -1 if the slot is free
+ *   last_use  int64 [slots]       tick of each slot's last use
+ * wanted (int32 [n_wanted], pages in [0, host_pages), duplicates allowed) are
+ * the pages of this step; keep (int32 [n_keep]) the pages of the step still in
+ * flight, which are never evicted.  Each distinct wanted page, in order of
+ * first occurrence: a resident page is a hit (its slot's last_use becomes
+ * tick); a missing page takes the next free slot in ascending order, then the
+ * least recently used slot (ties to the lower slot) whose page is neither
+ * wanted nor kept, evicting that page.
+ * Outputs (capacity `slots` entries each):
+ *   pairs    int32 [n][2] {host page, slot} of the missing pages, in order
+ *   evicted  int32 [m] host pages removed from their slots, in claim order
+ *   counts   int32 [4] {n, m, hits, distinct wanted pages}
+ * Errors: SA_ERR_INVALID_ARGUMENT (a null pointer, slots or host_pages < 1, a
+ * wanted or kept page out of range); SA_ERR_CAPACITY (more distinct wanted
+ * pages than slots, or too few slots that may be evicted).  On an error the
+ * state arrays are left unchanged.  Thread-safe for distinct state arrays.
+ */
+SA_API sa_status sa_tier_plan(int32_t *slot_of, int64_t host_pages, int32_t *page_in, int64_t *last_use,
+                              int32_t slots, int64_t tick, const int32_t *wanted, int32_t n_wanted,
+                              const int32_t *keep, int32_t n_keep, int32_t *pairs, int32_t *evicted,
+                              int32_t *counts);
+
+/* ------------------------------------------------------------------------ */
 /* Workspace sizing, status                                                 */
 /* ------------------------------------------------------------------------ */
 typedef enum {

@@ -23,7 +23,7 @@ OP_SELECT_TOPK, OP_SELECT_BLOCKS, OP_DECODE, OP_PREFILL = 1, 2, 3, 4
 
 EXPORTS = ("sa_select_topk", "sa_select_blocks", "sa_sparse_decode_attn", "sa_sparse_prefill_attn",
            "sa_workspace_bytes", "sa_workspace_init", "sa_read_device_status", "sa_status_string",
-           "sa_version", "sa_sparse_decode_attn_noalloc", "sa_fetch_pages")
+           "sa_version", "sa_sparse_decode_attn_noalloc", "sa_fetch_pages", "sa_tier_plan")
 
 
 class KVCacheS(ctypes.Structure):
@@ -79,6 +79,8 @@ def load(path: str = LIB_PATH):
                                  c_vp, c_size, c_vp]
     L.sa_sparse_prefill_attn.argtypes = [P(KVCacheS), c_vp, c_i32, c_i32, P(BlockListS), c_f32, c_i32,
                                          c_vp, c_vp, c_vp, c_size, c_vp]
+    L.sa_tier_plan.argtypes = [c_vp, ctypes.c_int64, c_vp, c_vp, c_i32, ctypes.c_int64, c_vp, c_i32, c_vp, c_i32,
+                               c_vp, c_vp, c_vp]
     L.sa_workspace_bytes.argtypes = [c_i32, P(KVCacheS), P(WsQueryS)]
     L.sa_workspace_bytes.restype = c_size
     L.sa_workspace_init.argtypes = [c_vp, c_size, c_vp]
@@ -87,7 +89,8 @@ def load(path: str = LIB_PATH):
     L.sa_status_string.restype = ctypes.c_char_p
     L.sa_version.restype = c_i32
     for fn in ("sa_select_topk", "sa_select_blocks", "sa_sparse_decode_attn", "sa_sparse_prefill_attn",
-               "sa_workspace_init", "sa_read_device_status", "sa_sparse_decode_attn_noalloc", "sa_fetch_pages"):
+               "sa_workspace_init", "sa_read_device_status", "sa_sparse_decode_attn_noalloc", "sa_fetch_pages",
+               "sa_tier_plan"):
         getattr(L, fn).restype = c_i32
     _lib = L
     return L

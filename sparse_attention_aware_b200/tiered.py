@@ -25,22 +25,40 @@ from typing import Iterable, List, Optional, Sequence, Set, Tuple
 import numpy as np
 import torch
 
-from . import api
+from . import _lib, api
 from .cache import PagedCache
+
+_CAPACITY = 7   # SA_ERR_CAPACITY
+
+
+def span_page_ranges(spans: Sequence[Tuple[int, int, bool]], seq_len: int,
+                     page_size: int) -> List[Tuple[int, int]]:
+    """The pages ``span_pages`` lists, as ascending disjoint ranges [lo, hi)."""
+    iv = []
+    for a, b, _ in spans:
+        a, b = max(a, 0), min(b, seq_len)
+        if a < b:
+            iv.append((a // page_size, (b - 1) // page_size + 1))
+    if not iv:
+        return []
+    iv.sort()
+    out: List[Tuple[int, int]] = []
+    lo, hi = iv[0]
+    for x, y in iv[1:]:
+        if x > hi:
+            out.append((lo, hi))
+            lo, hi = x, y
+        elif y > hi:
+            hi = y
+    out.append((lo, hi))
+    return out
 
 
 def span_pages(spans: Sequence[Tuple[int, int, bool]], seq_len: int, page_size: int) -> List[int]:
     """Logical pages a step reads for one sequence's span list: every page a
     span touches after clipping to [0, seq_len) (rounding a span out to page
-    edges does not change the pages it touches), ascending."""
-    parts = []
-    for a, b, _ in spans:
-        a, b = max(a, 0), min(b, seq_len)
-        if a < b:
-            parts.append(np.arange(a // page_size, (b - 1) // page_size + 1))
-    if not parts:
-        return []
-    return np.unique(np.concatenate(parts)).tolist()
+    edges does not change the pages it touches), ascending, each once."""
+    return [p for lo, hi in span_page_ranges(spans, seq_len, page_size) for p in range(lo, hi)]
 
 
 class SlotMap:
@@ -50,58 +68,52 @@ class SlotMap:
     missing pages take free slots first, then the least recently used slots
     whose pages neither this step nor the step still in flight reads (by
     default the previous ``plan``'s pages).  It returns the (host page, slot)
-    fetches and raises if the pool cannot hold the step."""
+    fetches and raises if the pool cannot hold the step.  The planning itself
+    is ``sa_tier_plan`` in libsa (host code), over this object's arrays."""
 
     def __init__(self, host_pages: int, slots: int):
         if slots <= 0:
             raise ValueError("need at least one device slot")
         self.slots = slots
-        self.slot_of = np.full(host_pages, -1, dtype=np.int64)   # host page -> slot
-        self.page_in = np.full(slots, -1, dtype=np.int64)        # slot -> host page
+        self.slot_of = np.full(host_pages, -1, dtype=np.int32)   # host page -> slot
+        self.page_in = np.full(slots, -1, dtype=np.int32)        # slot -> host page
         self.last_use = np.full(slots, -1, dtype=np.int64)
         self.tick = 0
-        self.prev = np.zeros(0, dtype=np.int64)
+        self.prev = np.zeros(0, dtype=np.int32)
         self.evicted: List[int] = []   # host pages the last plan evicted
         self.stats = {"hits": 0, "misses": 0}
+        self._pairs = np.zeros((slots, 2), dtype=np.int32)
+        self._ev = np.zeros(slots, dtype=np.int32)
+        self._counts = np.zeros(4, dtype=np.int32)
+        # the state arrays never move: their addresses once
+        self._ptrs = tuple(x.ctypes.data for x in (self.slot_of, self.page_in, self.last_use, self._pairs,
+                                                     self._ev, self._counts))
+
+    def plan_array(self, wanted, in_flight: Optional[Set[int]] = None) -> np.ndarray:
+        """``plan`` returning the fetches as an int32 array [n][2] (a view,
+        valid until the next call)."""
+        w = np.ascontiguousarray(np.asarray(wanted).ravel(), dtype=np.int32)
+        keep = self.prev if in_flight is None else np.asarray(sorted(in_flight), dtype=np.int32)
+        keep = np.ascontiguousarray(keep, dtype=np.int32)
+        self.tick += 1
+        ps, pp, pl, pa, pe, pc = self._ptrs
+        st = _lib.load().sa_tier_plan(ps, len(self.slot_of), pp, pl, self.slots, self.tick,
+                                      w.__array_interface__["data"][0], len(w),
+                                      keep.__array_interface__["data"][0], len(keep), pa, pe, pc)
+        if st == _CAPACITY:
+            raise RuntimeError("the pages of this step (%d distinct) and of the step in flight do not fit the "
+                               "device pool of %d slots" % (len(np.unique(w)), self.slots))
+        if st != _lib.SA_OK:
+            raise ValueError("sa_tier_plan: %s" % _lib.STATUS_NAMES.get(st, st))
+        n, m, hits, _ = (int(x) for x in self._counts)
+        self.stats["hits"] += hits
+        self.stats["misses"] += n
+        self.evicted = self._ev[:m].tolist()
+        self.prev = w
+        return self._pairs[:n]
 
     def plan(self, wanted: Sequence[int], in_flight: Optional[Set[int]] = None) -> List[Tuple[int, int]]:
-        self.tick += 1
-        w = np.asarray(wanted, dtype=np.int64).ravel()
-        _, first = np.unique(w, return_index=True)
-        w = w[np.sort(first)]                      # distinct, in first-occurrence order
-        if len(w) > self.slots:
-            raise RuntimeError("step needs %d pages, the device pool has %d slots" % (len(w), self.slots))
-        prev = self.prev if in_flight is None else np.asarray(sorted(in_flight), dtype=np.int64)
-        keep = np.union1d(w, prev)
-        slots_w = self.slot_of[w]
-        hit = slots_w >= 0
-        self.last_use[slots_w[hit]] = self.tick
-        self.stats["hits"] += int(hit.sum())
-        missing = w[~hit]
-        pairs = []
-        self.evicted = []
-        if len(missing):
-            free = np.nonzero(self.page_in < 0)[0]
-            cand = free
-            if len(free) < len(missing):
-                used = np.nonzero((self.page_in >= 0) & ~np.isin(self.page_in, keep))[0]
-                used = used[np.lexsort((used, self.last_use[used]))]
-                cand = np.concatenate([free, used[: len(missing) - len(free)]])
-            if len(cand) < len(missing):
-                raise RuntimeError("not enough evictable slots: the pages of this step and of the step in "
-                                   "flight exceed the device pool")
-            cand = cand[: len(missing)]
-            old = self.page_in[cand]
-            ev = old[old >= 0]
-            self.slot_of[ev] = -1
-            self.evicted = ev.tolist()
-            self.page_in[cand] = missing
-            self.slot_of[missing] = cand
-            self.last_use[cand] = self.tick
-            pairs = list(zip(missing.tolist(), cand.tolist()))
-            self.stats["misses"] += len(missing)
-        self.prev = w
-        return pairs
+        return [(int(p), int(s)) for p, s in self.plan_array(wanted, in_flight)]
 
 
 class TieredKV:
@@ -171,8 +183,20 @@ class TieredKV:
         return self.host_k[0].numel() * 2
 
     def host_pages_of(self, need: Sequence[Iterable[int]]) -> np.ndarray:
-        parts = [self.host_pt[b, np.asarray(pages, dtype=np.int64)] for b, pages in enumerate(need) if len(pages)]
-        return np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
+        lens = [len(p) for p in need]
+        lp = np.fromiter((x for pages in need for x in pages), dtype=np.int64, count=sum(lens))
+        b = np.repeat(np.arange(len(need), dtype=np.int64), lens)
+        return self.host_pt[b, lp]
+
+    def prepare_spans(self, span_lists: Sequence[Sequence[Tuple[int, int, bool]]], seq_lens: Sequence[int],
+                      compute_stream: Optional[torch.cuda.Stream] = None) -> int:
+        """``prepare`` for the pages of per-sequence span lists (the pages
+        ``span_pages(span_lists[b], seq_lens[b], P)`` names), mapped through
+        the host page table range by range."""
+        parts = [self.host_pt[b, lo:hi] for b, (spans, n) in enumerate(zip(span_lists, seq_lens))
+                 for lo, hi in span_page_ranges(spans, n, self.P)]
+        wanted = np.concatenate(parts) if parts else np.zeros(0, dtype=np.int64)
+        return self._prepare_pages(wanted, compute_stream, seq_lens)
 
     def prepare(self, need: Sequence[Iterable[int]], compute_stream: Optional[torch.cuda.Stream] = None,
                 seq_lens: Optional[Sequence[int]] = None) -> int:
@@ -187,19 +211,21 @@ class TieredKV:
         same ones (``span_pages(spans, seq_lens[b], P)``): a span that reaches
         past the length the host clipped to would make the device read a page
         that was never requested."""
+        return self._prepare_pages(self.host_pages_of(need), compute_stream, seq_lens)
+
+    def _prepare_pages(self, wanted: np.ndarray, compute_stream, seq_lens) -> int:
         compute_stream = compute_stream or torch.cuda.current_stream(self.device)
         # the step queued just before this call may still be running and its
         # pages are kept; older steps must be done before a slot is reused
         mark = torch.cuda.Event()
         mark.record(compute_stream)
-        pairs = self.map.plan(self.host_pages_of(need))
-        changed = bool(pairs)
+        pairs = self.map.plan_array(wanted)
+        changed = len(pairs) > 0
         if self.map.evicted:
             ev = np.asarray(self.map.evicted)
             self.pt[self.where_b[ev], self.where_lp[ev]] = -1
-        if pairs:
-            pa = np.asarray(pairs)
-            self.pt[self.where_b[pa[:, 0]], self.where_lp[pa[:, 0]]] = pa[:, 1]
+        if changed:
+            self.pt[self.where_b[pairs[:, 0]], self.where_lp[pairs[:, 0]]] = pairs[:, 1]
         lbuf = self.lens_cur ^ 1
         if seq_lens is not None:
             if len(seq_lens) != self.host_pt.shape[0]:
@@ -216,13 +242,13 @@ class TieredKV:
         with torch.cuda.stream(self.stream):
             if self.prev_mark is not None:
                 self.stream.wait_event(self.prev_mark)
-            if pairs:
+            if changed:
                 n = len(pairs)
                 hb = self.pflip
                 self.pflip ^= 1
                 if self.pairs_free[hb] is not None:
                     self.pairs_free[hb].synchronize()     # its copy two fetches ago is done
-                self.pairs_host[hb].numpy()[:n] = np.asarray(pairs, dtype=np.int32)
+                self.pairs_host[hb].numpy()[:n] = pairs
                 pr = self.pairs_dev[:n]
                 pr.copy_(self.pairs_host[hb][:n], non_blocking=True)
                 done_p = torch.cuda.Event()

@@ -78,7 +78,10 @@ def test_tiered_masked_decode_is_bitwise_the_resident_decode(cuda_dev):
             m.observe(streams[b][i])
             lists.append(m.next_spans(lens[b]))
         spans, cnt, rnd = SP.pack(lists, cuda_dev, max_spans=2)
-        fetched += tier.prepare([T.span_pages(l, L, P) for l, L in zip(lists, lens)], seq_lens=lens)
+        if i % 2:   # both entry points: page lists, and span lists mapped range by range
+            fetched += tier.prepare_spans(lists, lens)
+        else:
+            fetched += tier.prepare([T.span_pages(l, L, P) for l, L in zip(lists, lens)], seq_lens=lens)
         tc = tier.cache
         assert torch.equal(tc.seq_lens, lens_t)
         rc = W.PagedCache(res.k, res.v, res.page_table, lens_t)

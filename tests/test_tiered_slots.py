@@ -1,5 +1,6 @@
 """Tiered KV host bookkeeping (CPU): residency, LRU eviction, pages of the
 step in flight never evicted, capacity errors, span -> page sets."""
+import numpy as np
 import pytest
 
 from sparse_attention_aware_b200 import tiered as T
@@ -47,3 +48,90 @@ def test_span_pages():
     assert T.span_pages([(0, 4, False), (5000, 6024, False)], 6000, 16) == [0] + list(range(312, 375))
     assert T.span_pages([(-100, 20, True), (15, 33, True)], 30, 16) == [0, 1]
     assert T.span_pages([(40, 40, True), (90, 120, True)], 64, 16) == []
+
+
+def _reference_plan(state, wanted, keep):
+    """The planning rule written out with numpy (test reference): distinct
+    wanted pages in first-occurrence order; hits refresh their slot's tick;
+    missing pages take free slots (ascending), then the least recently used
+    slots (ties to the lower slot) whose page is neither wanted nor kept."""
+    slot_of, page_in, last_use, tick = state
+    w = np.asarray(wanted, dtype=np.int64)
+    _, first = np.unique(w, return_index=True)
+    w = w[np.sort(first)]
+    if len(w) > len(page_in):
+        return None
+    keep_all = np.union1d(w, np.asarray(keep, dtype=np.int64))
+    sl = slot_of[w]
+    missing = w[sl < 0]
+    free = np.nonzero(page_in < 0)[0]
+    cand = free
+    if len(free) < len(missing):
+        used = np.nonzero((page_in >= 0) & ~np.isin(page_in, keep_all))[0]
+        used = used[np.lexsort((used, last_use[used]))]
+        cand = np.concatenate([free, used[: len(missing) - len(free)]])
+    if len(cand) < len(missing):
+        return None
+    last_use[sl[sl >= 0]] = tick
+    cand = cand[: len(missing)]
+    old = page_in[cand]
+    ev = old[old >= 0]
+    slot_of[ev] = -1
+    page_in[cand] = missing
+    slot_of[missing] = cand
+    last_use[cand] = tick
+    return list(zip(missing.tolist(), cand.tolist())), ev.tolist(), int((sl >= 0).sum())
+
+
+def test_native_plan_matches_the_rule_on_random_streams():
+    rng = np.random.default_rng(7)
+    for trial in range(20):
+        host_pages, slots = int(rng.integers(20, 400)), int(rng.integers(4, 64))
+        m = T.SlotMap(host_pages, slots)
+        ref = (np.full(host_pages, -1, np.int64), np.full(slots, -1, np.int64), np.full(slots, -1, np.int64), 0)
+        prev = []
+        for step in range(40):
+            n = int(rng.integers(0, slots + 3))
+            base = int(rng.integers(0, host_pages))
+            wanted = ((base + rng.integers(0, max(1, 2 * slots), n)) % host_pages).tolist()
+            inflight = None if rng.random() < 0.7 else set(rng.integers(0, host_pages, 3).tolist())
+            keep = prev if inflight is None else sorted(inflight)
+            tick = step + 1
+            ref_state = (ref[0], ref[1], ref[2], tick)
+            before = (ref[0].copy(), ref[1].copy(), ref[2].copy())
+            want = _reference_plan(ref_state, wanted, keep)
+            if want is None:
+                with pytest.raises(RuntimeError):
+                    m.plan(wanted, in_flight=inflight)
+                ref = (before[0], before[1], before[2], tick)
+                # the native call leaves the state unchanged on a capacity error
+                np.testing.assert_array_equal(m.slot_of, before[0])
+                np.testing.assert_array_equal(m.page_in, before[1])
+                m.prev = np.asarray(prev, dtype=np.int32) if inflight is None else m.prev
+                continue
+            pairs, ev, hits = want
+            hits0 = m.stats["hits"]
+            assert m.plan(wanted, in_flight=inflight) == pairs
+            assert m.evicted == ev and m.stats["hits"] - hits0 == hits
+            np.testing.assert_array_equal(m.slot_of, ref[0])
+            np.testing.assert_array_equal(m.page_in, ref[1])
+            np.testing.assert_array_equal(m.last_use, ref[2])
+            prev = wanted
+
+
+def test_native_plan_rejects_bad_pages():
+    m = T.SlotMap(10, 2)
+    with pytest.raises(ValueError):
+        m.plan([10])
+    with pytest.raises(ValueError):
+        m.plan([-1])
+
+
+def test_span_pages_matches_the_set_definition():
+    rng = np.random.default_rng(3)
+    for _ in range(200):
+        L, P = int(rng.integers(1, 5000)), int(rng.choice([16, 64]))
+        spans = [(int(a), int(a + rng.integers(-50, 900)), bool(rng.integers(0, 2)))
+                 for a in rng.integers(-100, L + 100, int(rng.integers(0, 4)))]
+        want = sorted({t // P for a, b, _ in spans for t in range(max(a, 0), min(b, L))})
+        assert T.span_pages(spans, L, P) == want
