@@ -510,7 +510,7 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
     pdl_trigger();
     __shared__ uint32_t bits[kSchedRows][kSchedWords + 1];   // +1: conflict-free column reads
     __shared__ int cost[kSchedPairs];
-    __shared__ int red_c[8], red_p[8];
+    __shared__ int red_c[2][8], red_p[2][8];   // double-buffered by iteration
     __shared__ int pr_a[kSchedRows / 2], pr_b[kSchedRows / 2];
     __shared__ int s_best[kSchedRows], s_taken;
     __shared__ unsigned long long s_used;
@@ -586,23 +586,37 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
     for (int round = 0; round < kSchedRows; ++round) {
         const unsigned long long u = s_used;
         if (s_taken >= nc / 2) break;   // uniform: read after a barrier
-        for (int ka = warp; ka < nc; ka += 8) {
-            uint32_t bk = 0xFFFFFFFFu;
-            if (!(u >> ka & 1ull)) {
-                for (int kb = lane; kb < nc; kb += 32) {
-                    if (kb == ka || (u >> kb & 1ull)) continue;
-                    const int lo = min(ka, kb), hi = max(ka, kb);
-                    const uint32_t key =
-                        ((uint32_t)min(cost[pair_index(lo, hi, nc)], (1 << 20) - 1) << 12) | (lo << 6) | hi;
-                    bk = min(bk, key);
+        // each warp's rows ka = warp + 8 j, all eight reduced together so that
+        // their shuffle chains overlap; lanes scan the partners kb = lane, lane + 32
+        uint32_t bk[kSchedRows / 8];
+#pragma unroll
+        for (int j = 0; j < kSchedRows / 8; ++j) {
+            const int ka = warp + 8 * j;
+            bk[j] = 0xFFFFFFFFu;
+            if (ka < nc && !(u >> ka & 1ull)) {
+#pragma unroll
+                for (int hh = 0; hh < 2; ++hh) {
+                    const int kb = lane + 32 * hh;
+                    if (kb < nc && kb != ka && !(u >> kb & 1ull)) {
+                        const int lo = min(ka, kb), hi = max(ka, kb);
+                        const uint32_t key =
+                            ((uint32_t)min(cost[pair_index(lo, hi, nc)], (1 << 20) - 1) << 12) | (lo << 6) | hi;
+                        bk[j] = min(bk[j], key);
+                    }
                 }
             }
+        }
 #pragma unroll
-            for (int o = 16; o > 0; o >>= 1) bk = min(bk, __shfl_xor_sync(0xffffffffu, bk, o));
-            if (lane == 0) {
-                const int lo = (bk >> 6) & 63, hi = bk & 63;
-                s_best[ka] = bk == 0xFFFFFFFFu ? -1 : (lo == ka ? hi : lo);
-            }
+        for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+            for (int j = 0; j < kSchedRows / 8; ++j) bk[j] = min(bk[j], __shfl_xor_sync(0xffffffffu, bk[j], o));
+        uint32_t mine = bk[0];
+#pragma unroll
+        for (int j = 1; j < kSchedRows / 8; ++j)
+            if (lane == j) mine = bk[j];
+        if (lane < kSchedRows / 8 && warp + 8 * lane < nc) {
+            const int ka = warp + 8 * lane, lo = (mine >> 6) & 63, hi = mine & 63;
+            s_best[ka] = mine == 0xFFFFFFFFu ? -1 : (lo == ka ? hi : lo);
         }
         __syncthreads();
         if (warp == 0) {
@@ -697,19 +711,19 @@ __global__ void __launch_bounds__(256) k_prefill_schedule_window(const PrefillAr
                 bq = oq;
             }
         }
+        const int rb = it & 1;           // this iteration's buffer: the next one writes the other
         if (lane == 0) {
-            red_c[warp] = bg;
-            red_p[warp] = bq;
+            red_c[rb][warp] = bg;
+            red_p[rb][warp] = bq;
         }
         __syncthreads();
-        bg = red_c[0];
-        bq = red_p[0];
+        bg = red_c[rb][0];
+        bq = red_p[rb][0];
         for (int w = 1; w < 8; ++w)
-            if (red_c[w] > bg || (red_c[w] == bg && red_p[w] < bq)) {
-                bg = red_c[w];
-                bq = red_p[w];
+            if (red_c[rb][w] > bg || (red_c[rb][w] == bg && red_p[rb][w] < bq)) {
+                bg = red_c[rb][w];
+                bq = red_p[rb][w];
             }
-        __syncthreads();                 // every thread has read red_*
         if (bg <= 0) break;              // uniform: every thread reduced the same values
         if (tid == 0) {
             const int x = sw_x[bq >> 1], y = sw_y[bq >> 1];
