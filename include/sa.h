@@ -370,15 +370,24 @@ SA_API sa_status sa_fetch_pages(const void *host_k, const void *host_v, void *de
  *   pairs    int32 [n][2] {host page, slot} of the missing pages, in order
  *   evicted  int32 [m] host pages removed from their slots, in claim order
  *   counts   int32 [4] {n, m, hits, distinct wanted pages}
+ *   scratch  int32 [scratch_ints], scratch_ints >= sa_tier_plan_scratch_ints(
+ *            host_pages, slots); zero-filled before the first call and then
+ *            kept with the state arrays (it holds the page marks between
+ *            calls); the library allocates nothing and keeps no state.
  * Errors: SA_ERR_INVALID_ARGUMENT (a null pointer, slots or host_pages < 1, a
- * wanted or kept page out of range); SA_ERR_CAPACITY (more distinct wanted
- * pages than slots, or too few slots that may be evicted).  On an error the
- * state arrays are left unchanged.  Thread-safe for distinct state arrays.
+ * wanted or kept page out of range); SA_ERR_WORKSPACE (scratch too small);
+ * SA_ERR_CAPACITY (more distinct wanted pages than slots, or too few slots that
+ * may be evicted).  On an error the state arrays are left unchanged.  Calls on
+ * distinct state and scratch arrays may run concurrently.
  */
 SA_API sa_status sa_tier_plan(int32_t *slot_of, int64_t host_pages, int32_t *page_in, int64_t *last_use,
                               int32_t slots, int64_t tick, const int32_t *wanted, int32_t n_wanted,
                               const int32_t *keep, int32_t n_keep, int32_t *pairs, int32_t *evicted,
-                              int32_t *counts);
+                              int32_t *counts, int32_t *scratch, int64_t scratch_ints);
+
+/* int32 words of scratch sa_tier_plan needs: 1 + host_pages + 4 * slots (0 if
+ * either argument is < 1). */
+SA_API int64_t sa_tier_plan_scratch_ints(int64_t host_pages, int32_t slots);
 
 /* ------------------------------------------------------------------------ */
 /* Workspace sizing, status                                                 */

@@ -85,9 +85,10 @@ class SlotMap:
         self._pairs = np.zeros((slots, 2), dtype=np.int32)
         self._ev = np.zeros(slots, dtype=np.int32)
         self._counts = np.zeros(4, dtype=np.int32)
+        self._scratch = np.zeros(int(_lib.load().sa_tier_plan_scratch_ints(host_pages, slots)), dtype=np.int32)
         # the state arrays never move: their addresses once
         self._ptrs = tuple(x.ctypes.data for x in (self.slot_of, self.page_in, self.last_use, self._pairs,
-                                                     self._ev, self._counts))
+                                                     self._ev, self._counts, self._scratch))
 
     def plan_array(self, wanted, in_flight: Optional[Set[int]] = None) -> np.ndarray:
         """``plan`` returning the fetches as an int32 array [n][2] (a view,
@@ -96,10 +97,11 @@ class SlotMap:
         keep = self.prev if in_flight is None else np.asarray(sorted(in_flight), dtype=np.int32)
         keep = np.ascontiguousarray(keep, dtype=np.int32)
         self.tick += 1
-        ps, pp, pl, pa, pe, pc = self._ptrs
+        ps, pp, pl, pa, pe, pc, px = self._ptrs
         st = _lib.load().sa_tier_plan(ps, len(self.slot_of), pp, pl, self.slots, self.tick,
                                       w.__array_interface__["data"][0], len(w),
-                                      keep.__array_interface__["data"][0], len(keep), pa, pe, pc)
+                                      keep.__array_interface__["data"][0], len(keep), pa, pe, pc,
+                                      px, len(self._scratch))
         if st == _CAPACITY:
             raise RuntimeError("the pages of this step (%d distinct) and of the step in flight do not fit the "
                                "device pool of %d slots" % (len(np.unique(w)), self.slots))

@@ -135,3 +135,34 @@ def test_span_pages_matches_the_set_definition():
                  for a in rng.integers(-100, L + 100, int(rng.integers(0, 4)))]
         want = sorted({t // P for a, b, _ in spans for t in range(max(a, 0), min(b, L))})
         assert T.span_pages(spans, L, P) == want
+
+
+def test_tier_plan_abi_scratch_and_errors():
+    """The C entry point directly: the scratch size formula, a short scratch
+    (SA_ERR_WORKSPACE), too many distinct pages (SA_ERR_CAPACITY) with the
+    state left unchanged, and a first call on a zero-filled scratch."""
+    from sparse_attention_aware_b200 import _lib
+    lib = _lib.load()
+    hp, slots = 50, 3
+    need = lib.sa_tier_plan_scratch_ints(hp, slots)
+    assert need == 1 + hp + 4 * slots and lib.sa_tier_plan_scratch_ints(0, slots) == 0
+    slot_of = np.full(hp, -1, np.int32)
+    page_in = np.full(slots, -1, np.int32)
+    last_use = np.full(slots, -1, np.int64)
+    pairs = np.zeros((slots, 2), np.int32)
+    ev = np.zeros(slots, np.int32)
+    counts = np.zeros(4, np.int32)
+    scratch = np.zeros(need, np.int32)
+
+    def call(wanted, scr=scratch, n_scr=None):
+        w = np.asarray(wanted, np.int32)
+        return lib.sa_tier_plan(slot_of.ctypes.data, hp, page_in.ctypes.data, last_use.ctypes.data, slots, 1,
+                                w.ctypes.data, len(w), None, 0, pairs.ctypes.data, ev.ctypes.data,
+                                counts.ctypes.data, scr.ctypes.data, need if n_scr is None else n_scr)
+
+    assert call([1], n_scr=need - 1) == 3                    # SA_ERR_WORKSPACE
+    assert call([1, 2, 3, 4]) == 7                          # SA_ERR_CAPACITY: 4 distinct > 3 slots
+    assert (slot_of == -1).all() and (page_in == -1).all()
+    assert call([4, 4, 9]) == 0
+    assert counts.tolist() == [2, 0, 0, 2] and pairs[:2].tolist() == [[4, 0], [9, 1]]
+    assert call([9, 4, 7, 9]) == 0 and counts.tolist() == [1, 0, 2, 3] and pairs[0].tolist() == [7, 2]
