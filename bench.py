@@ -409,6 +409,7 @@ def main():
     rbs_quant_ms = qs.elapsed_time(qe) / 5
     da_us = da_state_cost(cfg, dev)
     tiered = tiered_measure(msk, cfg, dev)
+    mg_us, mg_bytes = masked_graph_measure(step, msk, cfg)
     total_ms = t_start.elapsed_time(t_end)
     parts = {"decode": 0.0, "masked": 0.0, "rbs_select": 0.0, "prefill": 0.0}
     per_step = {"decode": [], "prefill": []}
@@ -475,7 +476,12 @@ def main():
         "masked_decode": {"ms_per_step": round(msk_ms / K, 4),
                           "gbs": round(world * msk_bytes / (msk_ms * 1e-3) / 1e9, 2),
                           "frac_hbm": round(msk_bytes / (msk_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
-                          "da_state_host_us_per_step": round(da_us, 2)},
+                          "da_state_host_us_per_step": round(da_us, 2),
+                          "graph": ({"us_per_step": round(mg_us, 2),
+                                     "gbs": round(mg_bytes / (mg_us * 1e-6) / 1e9, 2),
+                                     "frac_hbm": round(mg_bytes / (mg_us * 1e-6) / 1e9 / pk["hbm_gbs"], 4),
+                                     "note": "64 steps captured once in a CUDA graph and replayed (per rank)"}
+                                    if mg_us is not None else {"unavailable": mg_bytes})},
         "tiered_kv": tiered,
         "roofline": {"bound": "tensor", "kernel": "k_prefill_tc", "achieved": round(per_gpu_pre, 2),
                      "peak": pk["bf16_tflops"], "unit": "TFLOP/s",
@@ -508,6 +514,47 @@ def main():
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
+
+
+def masked_graph_measure(step, msk, cfg, steps=64, reps=5):
+    """The masked-decode step the way a launch-bound decode loop runs it: the
+    64 steps of the workload (span selection + decode + combine each) captured
+    once in a CUDA graph (the kernels' PDL edges included) and replayed;
+    device time per step from CUDA events around the replays.  Returns
+    (us per step, bytes per step) or (None, reason)."""
+    import torch
+    m = cfg.msk
+    qs = msk.q_steps
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    try:
+        with torch.cuda.stream(stream):
+            for s in range(steps):   # eager pass: every buffer has its size before the capture
+                step.mstep = s
+                step.masked_decode(qs[s % qs.shape[0]])
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            for s in range(steps):
+                step.mstep = s
+                step.masked_decode(qs[s % qs.shape[0]])
+    except Exception as e:   # reported, not fatal: the timed numbers above stand
+        return None, "capture failed: %s" % str(e).splitlines()[0][:120]
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    step.ws[1].raise_on_fault("masked decode graph")
+    us = e0.elapsed_time(e1) * 1000 / (reps * steps)
+    nbytes = sum(step.masked_tokens[s % len(step.masked_tokens)] for s in range(steps)) * m["Hkv"] * m["d"] * 4 \
+        / steps + 2 * m["B"] * m["Hq"] * m["d"] * 2
+    del g
+    return us, nbytes
 
 
 def tiered_measure(msk, cfg, dev, steps=64, slot_frac=0.125):
