@@ -418,6 +418,15 @@ SA_API size_t sa_workspace_bytes(sa_op op, const sa_kv_cache *kv, const sa_ws_qu
  * after allocating a workspace that was not zero-filled. */
 SA_API sa_status sa_workspace_init(void *ws, size_t ws_bytes, sa_stream_t stream);
 
+/* Diagnostic of the bounded waits: enqueues one CTA whose thread waits, with
+ * the bounded-wait helper every kernel uses, on an mbarrier that nothing ever
+ * arrives on.  After timeout_ns (0 < timeout_ns <= 1e10) the wait gives up,
+ * SA_ERR_TIMEOUT (check id 11, value -1) is recorded in ws as a kernel would
+ * record it, and the kernel returns; the context stays usable.
+ *   ws  any workspace of at least 256 bytes (only its status word is used).
+ * Errors: SA_ERR_INVALID_ARGUMENT (timeout out of range), SA_ERR_WORKSPACE. */
+SA_API sa_status sa_check_bounded_wait(int64_t timeout_ns, void *ws, size_t ws_bytes, sa_stream_t stream);
+
 /* Synchronises `stream`, then returns and clears the first error a kernel
  * recorded in `ws` (SA_OK if none).  detail (host, nullable) receives
  * {status, check id, offending value}. */

@@ -24,7 +24,7 @@ OP_SELECT_TOPK, OP_SELECT_BLOCKS, OP_DECODE, OP_PREFILL = 1, 2, 3, 4
 EXPORTS = ("sa_select_topk", "sa_select_blocks", "sa_sparse_decode_attn", "sa_sparse_prefill_attn",
            "sa_workspace_bytes", "sa_workspace_init", "sa_read_device_status", "sa_status_string",
            "sa_version", "sa_sparse_decode_attn_noalloc", "sa_fetch_pages", "sa_tier_plan",
-           "sa_tier_plan_scratch_ints")
+           "sa_tier_plan_scratch_ints", "sa_check_bounded_wait")
 
 
 class KVCacheS(ctypes.Structure):
@@ -82,6 +82,7 @@ def load(path: str = LIB_PATH):
                                          c_vp, c_vp, c_vp, c_size, c_vp]
     L.sa_tier_plan.argtypes = [c_vp, ctypes.c_int64, c_vp, c_vp, c_i32, ctypes.c_int64, c_vp, c_i32, c_vp, c_i32,
                                c_vp, c_vp, c_vp, c_vp, ctypes.c_int64]
+    L.sa_check_bounded_wait.argtypes = [ctypes.c_int64, c_vp, c_size, c_vp]
     L.sa_tier_plan_scratch_ints.argtypes = [ctypes.c_int64, c_i32]
     L.sa_tier_plan_scratch_ints.restype = ctypes.c_int64
     L.sa_workspace_bytes.argtypes = [c_i32, P(KVCacheS), P(WsQueryS)]
@@ -93,7 +94,7 @@ def load(path: str = LIB_PATH):
     L.sa_version.restype = c_i32
     for fn in ("sa_select_topk", "sa_select_blocks", "sa_sparse_decode_attn", "sa_sparse_prefill_attn",
                "sa_workspace_init", "sa_read_device_status", "sa_sparse_decode_attn_noalloc", "sa_fetch_pages",
-               "sa_tier_plan"):
+               "sa_tier_plan", "sa_check_bounded_wait"):
         getattr(L, fn).restype = c_i32
     _lib = L
     return L

@@ -292,6 +292,17 @@ def sparse_decode_attn(cache, q: torch.Tensor, sel, scale: Optional[float] = Non
 
 
 @_on_call_stream
+def check_bounded_wait(timeout_s: float, device=None, ws: Optional[Workspace] = None, stream=None) -> None:
+    """Enqueue the bounded-wait diagnostic (``sa_check_bounded_wait``): a wait
+    on an mbarrier that nothing arrives on gives up after ``timeout_s`` and
+    records SA_ERR_TIMEOUT in the workspace, which ``ws.status()`` then reads."""
+    dev = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
+    w = _ws(ws, dev, stream)
+    wp, wn = w.aligned(256, stream)
+    _check(L.load().sa_check_bounded_wait(int(timeout_s * 1e9), wp, wn, _stream(stream)), "sa_check_bounded_wait")
+
+
+@_on_call_stream
 def fetch_pages(host_k: torch.Tensor, host_v: torch.Tensor, dev_k: torch.Tensor, dev_v: torch.Tensor,
                 pairs: torch.Tensor, ws: Optional[Workspace] = None, stream=None) -> None:
     """Copy host-tier pages into device page slots (``sa_fetch_pages``).

@@ -184,6 +184,15 @@ sa_status sa_workspace_init(void *ws, size_t ws_bytes, sa_stream_t stream)
     return cuda_status(cudaMemsetAsync(ws, 0, kHeader, (cudaStream_t)stream));
 }
 
+sa_status sa_check_bounded_wait(int64_t timeout_ns, void *ws, size_t ws_bytes, sa_stream_t stream)
+{
+    if (timeout_ns <= 0 || timeout_ns > 10000000000ll) return SA_ERR_INVALID_ARGUMENT;
+    sa_status st = check_ws(ws, ws_bytes, kHeader);
+    if (st != SA_OK) return st;
+    return cuda_status(sa::launch_wait_diag(static_cast<DevStatus *>(ws), (unsigned long long)timeout_ns,
+                                            (cudaStream_t)stream));
+}
+
 sa_status sa_read_device_status(void *ws, sa_stream_t stream, int32_t *detail)
 {
     if (!ws || !aligned(ws, kAlign)) return SA_ERR_WORKSPACE;

@@ -73,6 +73,8 @@ struct TopkArgs {
     DevStatus *st;
 };
 cudaError_t launch_topk(const TopkArgs &a, cudaStream_t s);
+// diagnostic bounded wait (k_diag.cu)
+cudaError_t launch_wait_diag(DevStatus *st, unsigned long long timeout_ns, cudaStream_t s);
 
 // ---- spans ------------------------------------------------------------------
 struct SpanArgs {
