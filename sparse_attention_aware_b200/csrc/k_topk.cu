@@ -425,52 +425,43 @@ __global__ void __launch_bounds__(kSelThreads, 2) k_topk_select(const TopkArgs a
     const uint32_t D1 = prefix >> 21;
 
     // pass 2: bitmap of top digit > D1, candidates with top digit == D1.  A
-    // lane holds 4 consecutive entries, so 8 lanes make one 32-bit bitmap
-    // word: each lane's 4-bit nibble is shifted into place and OR-ed across
-    // the 8 lanes with xor shuffles.
+    // lane holds 8 consecutive entries (two adjacent 16-byte loads), so 4
+    // lanes make one 32-bit bitmap word: each lane's byte is shifted into
+    // place and OR-ed across the 4 lanes with two xor shuffles.
     if (tid == 0) s_ncand = 0;
     __syncthreads();
-    for (int v0 = 0; v0 < nv; v0 += kSelThreads * 4) {
-        float4 x[4];
+    const int no = (L + 7) >> 3;   // octets of entries (the row buffer is a multiple of 16 long)
+    for (int o = tid; o - tid < no; o += kSelThreads) {
+        const float4 x0 = o < no ? __ldcg(row4 + 2 * o) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const float4 x1 = o < no ? __ldcg(row4 + 2 * o + 1) : make_float4(0.f, 0.f, 0.f, 0.f);
+        const int t = o * 8;
+        const uint32_t kk[8] = {f2key(x0.x), f2key(x0.y), f2key(x0.z), f2key(x0.w),
+                                f2key(x1.x), f2key(x1.y), f2key(x1.z), f2key(x1.w)};
+        uint32_t hb = 0, eb = 0;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int v = v0 + u * kSelThreads + tid;
-            x[u] = v < nv ? __ldcg(row4 + v) : make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = 0; j < 8; ++j) {
+            const bool in = t + j < L;
+            const uint32_t dg = kk[j] >> 21;
+            hb |= (uint32_t)(in && dg > D1) << j;
+            eb |= (uint32_t)(in && dg == D1) << j;
         }
+        uint32_t hw = hb << (8 * (lane & 3));
+        hw |= __shfl_xor_sync(0xffffffffu, hw, 1);
+        hw |= __shfl_xor_sync(0xffffffffu, hw, 2);
+        if ((lane & 3) == 0 && (o >> 2) < nw) {
+            above[o >> 2] = hw;
+            eqmap[o >> 2] = 0u;
+        }
+        if (eb) {
+            unsigned slot = atomicAdd(&s_ncand, (unsigned)__popc(eb));
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int v = v0 + u * kSelThreads + tid;
-            const int t = v * 4;
-            const uint32_t kk[4] = {f2key(x[u].x), f2key(x[u].y), f2key(x[u].z), f2key(x[u].w)};
-            uint32_t hn = 0, en = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                const bool in = t + j < L;
-                const uint32_t dg = kk[j] >> 21;
-                hn |= (uint32_t)(in && dg > D1) << j;
-                en |= (uint32_t)(in && dg == D1) << j;
-            }
-            uint32_t hw = hn << (4 * (lane & 7)), ew = en << (4 * (lane & 7));
-#pragma unroll
-            for (int o = 1; o < 8; o <<= 1) {
-                hw |= __shfl_xor_sync(0xffffffffu, hw, o);
-                ew |= __shfl_xor_sync(0xffffffffu, ew, o);
-            }
-            if ((lane & 7) == 0 && (v >> 3) < nw) {
-                above[v >> 3] = hw;
-                eqmap[v >> 3] = 0u;
-            }
-            if (en) {
-                unsigned slot = atomicAdd(&s_ncand, (unsigned)__popc(en));
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    if (en >> j & 1) {
-                        if (slot < kCandCap) {
-                            ckey[slot] = kk[j];
-                            cpos[slot] = (uint32_t)(t + j);
-                        }
-                        ++slot;
+            for (int j = 0; j < 8; ++j) {
+                if (eb >> j & 1) {
+                    if (slot < kCandCap) {
+                        ckey[slot] = kk[j];
+                        cpos[slot] = (uint32_t)(t + j);
                     }
+                    ++slot;
                 }
             }
         }
