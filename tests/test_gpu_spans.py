@@ -141,6 +141,8 @@ def test_masked_decode_full_size_steps(cuda_dev):
     (64, 32, 2, torch.bfloat16),     # 16 query heads per kv head (all MMA rows used)
     (128, 8, 1, torch.float32),      # fp32 query (high + low bf16 parts)
     (128, 32, 1, torch.bfloat16),    # 32 per kv head: per-head kernel
+    (128, 12, 1, torch.bfloat16),    # 12 per kv head: two 8-head column blocks, 4 padding heads
+    (64, 6, 2, torch.float32),       # 3 per kv head, fp32 query, 5 padding heads
 ])
 def test_masked_decode_group_shapes(cuda_dev, d, Hq, Hkv, qdt):
     lens = [700, 4100, 33, 2500]
