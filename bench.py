@@ -410,6 +410,7 @@ def main():
     da_us = da_state_cost(cfg, dev)
     tiered = tiered_measure(msk, cfg, dev)
     mg_us, mg_bytes = masked_graph_measure(step, msk, cfg)
+    dg_ms, dg_why = decode_graph_measure(step, dec)
     total_ms = t_start.elapsed_time(t_end)
     parts = {"decode": 0.0, "masked": 0.0, "rbs_select": 0.0, "prefill": 0.0}
     per_step = {"decode": [], "prefill": []}
@@ -461,7 +462,13 @@ def main():
                    "union_frac_hbm": round(K * union_bytes / (dec_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
                    "ms_per_group": round(dec_ms / K, 4), "bytes_per_group": dec_bytes,
                    "ms_p50": pct(per_step["decode"], 50), "ms_p95": pct(per_step["decode"], 95),
-                   "tokens_per_s": round(world * K * cfg.dec["B"] / (dec_ms * 1e-3), 1)},
+                   "tokens_per_s": round(world * K * cfg.dec["B"] / (dec_ms * 1e-3), 1),
+                   "graph": ({"ms_per_group": round(dg_ms, 4),
+                              "gbs": round(dec_bytes / (dg_ms * 1e-3) / 1e9, 2),
+                              "frac_hbm": round(dec_bytes / (dg_ms * 1e-3) / 1e9 / pk["hbm_gbs"], 4),
+                              "note": "cross-check: the group captured once in a CUDA graph and replayed (per rank); "
+                                      "value and frac_hbm above are the eager step's"}
+                             if dg_ms is not None else {"unavailable": dg_why})},
         "prefill": {"tflops": round(pre_tflops, 2), "frac_bf16_sustained": round(per_gpu_pre / pk["bf16_tflops_sustained"], 4),
                     "frac_bf16_burst": round(per_gpu_pre / pk["bf16_tflops"], 4),
                     "ms": round(pre_ms / K, 4), "ms_p50": pct(per_step["prefill"], 50),
@@ -555,6 +562,37 @@ def masked_graph_measure(step, msk, cfg, steps=64, reps=5):
         / steps + 2 * m["B"] * m["Hq"] * m["d"] * 2
     del g
     return us, nbytes
+
+
+def decode_graph_measure(step, dec, reps=10):
+    """Cross-check of the decode group's time: the group (top-k + the decode
+    layers, with their combines) captured once in a CUDA graph and replayed;
+    device time per group from CUDA events around the replays.  Returns ms per
+    group, or None with the reason if the capture failed."""
+    import torch
+    stream = torch.cuda.Stream()
+    stream.wait_stream(torch.cuda.current_stream())
+    try:
+        with torch.cuda.stream(stream):
+            step.decode_group(dec.q_layers)
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step.decode_group(dec.q_layers)
+    except Exception as e:   # reported, not fatal
+        return None, "capture failed: %s" % str(e).splitlines()[0][:120]
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(reps):
+        g.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    step.ws[0].raise_on_fault("decode group graph")
+    del g
+    return e0.elapsed_time(e1) / reps, None
 
 
 def tiered_measure(msk, cfg, dev, steps=64, slot_frac=0.125):
