@@ -22,7 +22,10 @@
 // lane; rows past the entry's end repeat its last row, so every piece is
 // 16 finite rows and its probability is 0 there) into the warp's kNST-stage
 // ring, rows padded to D*2 + 16 bytes so that 8-row ldmatrix reads hit 32
-// distinct banks; each stage completes on its own mbarrier.
+// distinct banks; each stage completes on its own mbarrier.  Every wait is
+// bounded (globaltimer deadline, shared abort flag): on expiry the warp
+// records SA_ERR_TIMEOUT, waits (bounded) for its copies still in flight and
+// leaves its loop.
 //
 // The contractions take the 16 tokens of a piece as the M rows and the
 // group's heads as the N columns of m16n8k16 (no padding rows for 8 heads):
@@ -278,7 +281,7 @@ __global__ void __launch_bounds__(kGThreads) k_decode_gqa_blocks(const DecodeArg
                                                                   deadline, abort_flag));
             if (!ok) {
                 *abort_flag = 1;
-                if (lane == 0) fault(st, CHK_WAIT, n);
+                if (lane == 0) record(st, SA_ERR_TIMEOUT, CHK_WAIT, n);
                 alive = false;
                 break;
             }

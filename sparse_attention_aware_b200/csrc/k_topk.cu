@@ -176,7 +176,7 @@ __global__ void __launch_bounds__(ScoreGeom<D, HPG>::THREADS) k_topk_score(const
             // memory is released
             *abort_flag = 1;
             if (lane == 0) {
-                fault(a.st, CHK_WAIT, issued);
+                record(a.st, SA_ERR_TIMEOUT, CHK_WAIT, issued);
                 const uint64_t dl = tc::globaltimer() + kScoreWaitNs;
                 volatile int zero = 0;
                 for (int j = max(0, issued - NS); j < issued; ++j)
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__(ScoreGeom<D, HPG>::THREADS) k_topk_score(const
         if (!ok) {
             // a copy never completed: record it and stop this warp
             *abort_flag = 1;
-            if (lane == 0) fault(a.st, CHK_WAIT, i);
+            if (lane == 0) record(a.st, SA_ERR_TIMEOUT, CHK_WAIT, i);
             break;
         }
         const uint8_t *stage = sm + s * Gm::STAGE + gl * 16;
