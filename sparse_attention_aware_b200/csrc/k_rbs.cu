@@ -308,10 +308,24 @@ __global__ void __launch_bounds__(512) k_qhist(const RbsArgs a, int pass)
     for (int i = threadIdx.x; i < nb; i += blockDim.x) hist[i] = 0;
     __syncthreads();
     const float *x = a.pair_sc + (size_t)arr * nP;
-    for (size_t t = t0 + threadIdx.x; t < t1; t += blockDim.x) {
-        const uint32_t key = f2key(__ldcs(x + t));
+    auto count = [&](float v) {
+        const uint32_t key = f2key(v);
         if ((key & pmask) == prefix) atomicAdd(&hist[(key >> shift) & (nb - 1)], 1u);
+    };
+    // 16-byte loads over the aligned middle of [t0, t1); an array need not
+    // start on a 16-byte boundary, so up to 3 scores at each end are read singly
+    const size_t head = min((size_t)((16u - ((uintptr_t)(x + t0) & 15u)) & 15u) / 4, t1 - t0);
+    const size_t ta = t0 + head, nv = (t1 - ta) / 4, tb = ta + 4 * nv;
+    if (threadIdx.x < head) count(__ldcs(x + t0 + threadIdx.x));
+    const float4 *x4 = reinterpret_cast<const float4 *>(x + ta);
+    for (size_t v = threadIdx.x; v < nv; v += blockDim.x) {
+        const float4 f = __ldcs(x4 + v);
+        count(f.x);
+        count(f.y);
+        count(f.z);
+        count(f.w);
     }
+    if (threadIdx.x < t1 - tb) count(__ldcs(x + tb + threadIdx.x));
     __syncthreads();
     uint32_t *gh = qhist_of(a, arr, pass);
     for (int i = threadIdx.x; i < nb; i += blockDim.x)
