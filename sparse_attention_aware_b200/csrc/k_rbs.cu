@@ -406,16 +406,16 @@ __global__ void __launch_bounds__(256) k_mask_scores(const RbsArgs a)
     const int words = rbs_mask_words(a.nB);
     const int nw = i / 32 + 1;
     int cnt = 0;
-    for (int w0 = 0; w0 < nw; w0 += 4) {
-        float vc[4], vr[4];
+    for (int w0 = 0; w0 < nw; w0 += 8) {   // 16 loads per lane in flight
+        float vc[8], vr[8];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
             const int j = (w0 + u) * 32 + lane;
             vc[u] = j <= i ? __ldcs(sc + j) : 0.f;
             vr[u] = j <= i ? __ldcs(sr + j) : 0.f;
         }
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
+        for (int u = 0; u < 8; ++u) {
             const int j = (w0 + u) * 32 + lane;
             const bool keep = j <= i && (vc[u] > tc || vr[u] > tr || (a.force_diag && j == i) ||
                                          (a.force_first && j == 0));
